@@ -1,0 +1,317 @@
+// ds_api.cu -- C ABI of libds.so: argument validation, launch planning and
+// kernel dispatch. Declarations and the full contract are in include/ds.h.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <atomic>
+#include <mutex>
+#include <unordered_map>
+
+#include "../../include/ds.h"
+#include "ds_decode_kernel.cuh"
+#include "ds_internal.h"
+
+namespace {
+
+thread_local char g_err[256] = "";
+std::atomic<int> g_cluster_override{0};
+
+ds_status fail(ds_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+ds_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(DS_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool kv_dtype_ok(ds_dtype t) { return t == DS_F32 || t == DS_BF16; }
+bool c_ok(int c, int d) { return (c == 8 || c == 16 || c == 32 || c == 64 || c == 128) && c <= d; }
+bool d_ok(int d) { return d == 64 || d == 128; }
+
+int group_tier(int G) { return G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : 8; }
+
+// Number of SMs of the current device (148 on B200); queried once per process.
+int sm_count() {
+    static int n = [] {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+        return v > 0 ? v : 148;
+    }();
+    return n;
+}
+
+constexpr int kMaxSmem = 227 * 1024;
+constexpr int kCtasPerSm = 2;  // __launch_bounds__(256, 2) -> <= 128 registers
+
+struct Plan {
+    int N, chunk, lay_chunk, per, smem;
+};
+
+int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+// Cluster size N (CTAs per (b, kv head) row): the largest power of two whose
+// grid (rows * N CTAs) still fits in one wave of resident CTAs, keeping at
+// least 256 tokens per CTA; rows beyond one wave use N = 1. A forced N
+// (ds_sparse_decode_set_cluster) overrides the choice when feasible.
+bool make_plan(int rows, int G, int s, int d, int c, int topk, bool dense, int slots, int forced,
+               Plan* out) {
+    const int GT = group_tier(G);
+    const bool select_all = dense || topk >= s;
+    const int k_eff = topk < s ? topk : s;
+    Plan best{0, 0, 0, 0, 0};
+    for (int N = 1; N <= 16; N *= 2) {
+        Plan p;
+        p.N = N;
+        p.chunk = round_up((s + N - 1) / N, 32);
+        if (p.chunk > ds::kMaxChunk) continue;
+        p.lay_chunk = dense ? 0 : p.chunk;
+        p.per = select_all ? 0 : (k_eff + N - 1) / N;
+        p.smem = ds::decode_smem_layout(GT, d, c, p.lay_chunk, p.per).total;
+        if (p.smem > kMaxSmem) continue;
+        if (forced) {
+            if (N == forced) { *out = p; return true; }
+            continue;
+        }
+        if (best.N == 0) best = p;  // smallest feasible
+        if ((long long)rows * N <= slots && (N == 1 || p.chunk >= 256)) best = p;
+    }
+    if (best.N == 0) return false;
+    *out = best;
+    return true;
+}
+
+std::mutex g_attr_mu;
+std::unordered_map<const void*, int> g_attr_smem;
+
+cudaError_t prepare_kernel(ds::DecodeKernel kern, int smem, int N) {
+    std::lock_guard<std::mutex> lk(g_attr_mu);
+    auto it = g_attr_smem.find(reinterpret_cast<const void*>(kern));
+    if (it != g_attr_smem.end() && it->second >= smem) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    (void)N;
+    g_attr_smem[reinterpret_cast<const void*>(kern)] = kMaxSmem;
+    return cudaSuccess;
+}
+
+ds::DecodeKernel pick_kernel(ds_dtype kvdt, bool int4, int d, int c, int GT) {
+    if (kvdt == DS_F32) return int4 ? ds::decode_kernel_f32_i4(d, c, GT) : ds::decode_kernel_f32_fp(d, c, GT);
+    return int4 ? ds::decode_kernel_bf16_i4(d, c, GT) : ds::decode_kernel_bf16_fp(d, c, GT);
+}
+
+ds_status launch_decode(ds::DecodeKernel kern, const ds::DecodeParams& p, int rows, const Plan& pl,
+                        cudaStream_t st) {
+    cudaError_t e = prepare_kernel(kern, pl.smem, pl.N);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(rows * pl.N), 1, 1);
+    cfg.blockDim = dim3(ds::kNT, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)pl.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)pl.N;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, p);
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    return DS_OK;
+}
+
+ds_status check_common(int b, int hq, int hkv, int s, int s_cap, int d, ds_dtype kvdt) {
+    if (b < 1 || hkv < 1 || hq < 1) return fail(DS_ERR_INVALID_ARG, "b, hq and hkv must be >= 1");
+    if (hq % hkv) return fail(DS_ERR_INVALID_ARG, "hq (%d) must be a multiple of hkv (%d)", hq, hkv);
+    if (hq / hkv > 8) return fail(DS_ERR_UNSUPPORTED, "hq/hkv = %d > 8", hq / hkv);
+    if (s < 1 || s > s_cap) return fail(DS_ERR_INVALID_ARG, "need 1 <= s (%d) <= s_cap (%d)", s, s_cap);
+    if (!d_ok(d)) return fail(DS_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", d);
+    if (!kv_dtype_ok(kvdt)) return fail(DS_ERR_UNSUPPORTED, "k/v dtype %d (supported: f32, bf16)", (int)kvdt);
+    if ((long long)b * hkv * (long long)s_cap * d >= (1ll << 40))
+        return fail(DS_ERR_UNSUPPORTED, "cache too large");
+    if ((long long)b * hkv > (1ll << 26)) return fail(DS_ERR_UNSUPPORTED, "too many rows");
+    return DS_OK;
+}
+
+ds_status check_label(ds_dtype kdt, ds_dtype label_dt, int c, int d, const void* label,
+                      const uint16_t* lscale, const uint16_t* lzero) {
+    if (!c_ok(c, d)) return fail(DS_ERR_UNSUPPORTED, "heavy channels c=%d (supported: 8,16,32,64,128; c <= d)", c);
+    if (!label) return fail(DS_ERR_INVALID_ARG, "label is NULL");
+    if (!aligned16(label)) return fail(DS_ERR_INVALID_ARG, "label not 16-byte aligned");
+    if (label_dt == DS_INT4) {
+        if (!lscale || !lzero) return fail(DS_ERR_INVALID_ARG, "4-bit label needs lscale and lzero");
+        if (!aligned16(lscale) || !aligned16(lzero)) return fail(DS_ERR_INVALID_ARG, "lscale/lzero not 16-byte aligned");
+    } else if (label_dt != kdt) {
+        return fail(DS_ERR_INVALID_ARG, "label dtype must equal the key dtype or be DS_INT4");
+    }
+    return DS_OK;
+}
+
+ds_status run_label(const void* k, ds_dtype kdt, const int32_t* idx, int b, int hkv, int t_begin,
+                    int t_end, int s_cap, int d, int c, void* label, ds_dtype label_dt,
+                    uint16_t* lscale, uint16_t* lzero, cudaStream_t st) {
+    ds_status r = check_common(b, hkv, hkv, t_end, s_cap, d, kdt);
+    if (r != DS_OK) return r;
+    if ((r = check_label(kdt, label_dt, c, d, label, lscale, lzero)) != DS_OK) return r;
+    if (!k || !idx) return fail(DS_ERR_INVALID_ARG, "k or idx is NULL");
+    if (!aligned16(k) || !aligned16(idx)) return fail(DS_ERR_INVALID_ARG, "k/idx not 16-byte aligned");
+    ds::LabelArgs a{k, kdt == DS_BF16, label_dt == DS_INT4, idx, b, hkv, t_begin, t_end, s_cap, d, c,
+                    label, lscale, lzero};
+    cudaError_t e = ds::launch_label(a, st);
+    if (e != cudaSuccess) return cuda_fail(e, "label launch");
+    return DS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ds_status_string(ds_status st) {
+    switch (st) {
+    case DS_OK: return "DS_OK";
+    case DS_ERR_INVALID_ARG: return "DS_ERR_INVALID_ARG";
+    case DS_ERR_UNSUPPORTED: return "DS_ERR_UNSUPPORTED";
+    case DS_ERR_CUDA: return "DS_ERR_CUDA";
+    case DS_ERR_WORKSPACE: return "DS_ERR_WORKSPACE";
+    }
+    return "DS_ERR_UNKNOWN";
+}
+
+const char* ds_last_error(void) { return g_err; }
+
+void ds_sparse_decode_set_cluster(int n) { g_cluster_override.store(n); }
+
+ds_status ds_calibrate_workspace_size(int n_samples, int hq, int hkv, int w, int s, int d,
+                                      size_t* bytes) {
+    if (!bytes) return fail(DS_ERR_INVALID_ARG, "bytes is NULL");
+    if (n_samples < 1 || hkv < 1 || hq < 1 || w < 1 || s < 1)
+        return fail(DS_ERR_INVALID_ARG, "sizes must be >= 1");
+    if (hq % hkv) return fail(DS_ERR_INVALID_ARG, "hq must be a multiple of hkv");
+    if (!d_ok(d)) return fail(DS_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", d);
+    *bytes = ds::calib_workspace_bytes(n_samples, hkv, d);
+    return DS_OK;
+}
+
+ds_status ds_calibrate_channels(const void* q_win, const void* k, ds_dtype dt, int n_samples,
+                                int hq, int hkv, int w, int s, int d, int c, float* ratio_out,
+                                int32_t* idx_out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    size_t need = 0;
+    ds_status r = ds_calibrate_workspace_size(n_samples, hq, hkv, w, s, d, &need);
+    if (r != DS_OK) return r;
+    if (!kv_dtype_ok(dt)) return fail(DS_ERR_UNSUPPORTED, "dtype %d (supported: f32, bf16)", (int)dt);
+    if (c < 1 || c > d) return fail(DS_ERR_INVALID_ARG, "need 1 <= c (%d) <= d (%d)", c, d);
+    if (hq / hkv * (long long)w > (1 << 20)) return fail(DS_ERR_UNSUPPORTED, "window too large");
+    if (!q_win || !k || !idx_out || !ws) return fail(DS_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(q_win) || !aligned16(k) || !aligned16(idx_out) || !aligned16(ws) ||
+        (ratio_out && !aligned16(ratio_out)))
+        return fail(DS_ERR_INVALID_ARG, "pointer not 16-byte aligned");
+    if (ws_bytes < need) return fail(DS_ERR_WORKSPACE, "workspace %zu B < required %zu B", ws_bytes, need);
+    ds::CalibArgs a{q_win, k, dt == DS_BF16, n_samples, hq, hkv, w, s, d, c, ratio_out, idx_out, ws};
+    cudaError_t e = ds::launch_calib(a, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "calibration launch");
+    return DS_OK;
+}
+
+ds_status ds_build_label_cache(const void* k, ds_dtype kdt, const int32_t* idx, int b, int hkv,
+                               int s, int s_cap, int d, int c, void* label, ds_dtype label_dt,
+                               uint16_t* lscale, uint16_t* lzero, cudaStream_t stream) {
+    return run_label(k, kdt, idx, b, hkv, 0, s, s_cap, d, c, label, label_dt, lscale, lzero, stream);
+}
+
+ds_status ds_append_label(const void* k, ds_dtype kdt, const int32_t* idx, int b, int hkv, int pos,
+                          int s_cap, int d, int c, void* label, ds_dtype label_dt, uint16_t* lscale,
+                          uint16_t* lzero, cudaStream_t stream) {
+    if (pos < 0 || pos >= s_cap) return fail(DS_ERR_INVALID_ARG, "need 0 <= pos (%d) < s_cap (%d)", pos, s_cap);
+    return run_label(k, kdt, idx, b, hkv, pos, pos + 1, s_cap, d, c, label, label_dt, lscale, lzero,
+                     stream);
+}
+
+ds_status ds_sparse_decode_plan(int b, int hq, int hkv, int s, int d, int c, int topk, ds_dtype kvdt,
+                                ds_dtype label_dt, int* cluster_out, int* chunk_out, int* smem_out) {
+    ds_status r = check_common(b, hq, hkv, s, s, d, kvdt);
+    if (r != DS_OK) return r;
+    if (!c_ok(c, d)) return fail(DS_ERR_UNSUPPORTED, "heavy channels c=%d", c);
+    if (label_dt != DS_INT4 && label_dt != kvdt) return fail(DS_ERR_INVALID_ARG, "label dtype");
+    if (topk < 1) return fail(DS_ERR_INVALID_ARG, "topk must be >= 1");
+    Plan pl;
+    if (!make_plan(b * hkv, hq / hkv, s, d, c, topk, false, kCtasPerSm * 148, g_cluster_override.load(), &pl))
+        return fail(DS_ERR_UNSUPPORTED, "no feasible launch plan (s too long for 16 CTAs per row)");
+    if (cluster_out) *cluster_out = pl.N;
+    if (chunk_out) *chunk_out = pl.chunk;
+    if (smem_out) *smem_out = pl.smem;
+    return DS_OK;
+}
+
+ds_status ds_sparse_decode(const void* q, const void* k, const void* v, ds_dtype kvdt,
+                           const void* label, ds_dtype label_dt, const uint16_t* lscale,
+                           const uint16_t* lzero, const int32_t* idx, int b, int hq, int hkv, int s,
+                           int s_cap, int d, int c, int topk, float sm_scale, void* out,
+                           ds_dtype out_dt, int32_t* sel_out, float* score_out, cudaStream_t stream) {
+    ds_status r = check_common(b, hq, hkv, s, s_cap, d, kvdt);
+    if (r != DS_OK) return r;
+    if ((r = check_label(kvdt, label_dt, c, d, label, lscale, lzero)) != DS_OK) return r;
+    if (topk < 1) return fail(DS_ERR_INVALID_ARG, "topk must be >= 1");
+    if (!q || !k || !v || !idx || !out) return fail(DS_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(out) ||
+        (sel_out && !aligned16(sel_out)) || (score_out && !aligned16(score_out)))
+        return fail(DS_ERR_INVALID_ARG, "pointer not 16-byte aligned");
+    if (!(out_dt == DS_F32 || (out_dt == DS_BF16 && kvdt == DS_BF16)))
+        return fail(DS_ERR_INVALID_ARG, "out dtype must be DS_F32 or (with bf16 k/v) DS_BF16");
+    if (!(sm_scale == sm_scale)) return fail(DS_ERR_INVALID_ARG, "sm_scale is NaN");
+    const int G = hq / hkv, GT = group_tier(G);
+    const int rows = b * hkv;
+    Plan pl;
+    if (!make_plan(rows, G, s, d, c, topk, false, kCtasPerSm * sm_count(), g_cluster_override.load(), &pl))
+        return fail(DS_ERR_UNSUPPORTED, "no feasible launch plan (s too long for 16 CTAs per row)");
+    ds::DecodeKernel kern = pick_kernel(kvdt, label_dt == DS_INT4, d, c, GT);
+    if (!kern) return fail(DS_ERR_UNSUPPORTED, "no kernel for d=%d c=%d G=%d", d, c, G);
+    ds::DecodeParams p{};
+    p.q = q; p.k = k; p.v = v; p.label = label; p.lscale = lscale; p.lzero = lzero; p.idx = idx;
+    p.out = out; p.sel_out = sel_out; p.score_out = score_out;
+    p.hkv = hkv; p.G = G; p.s = s; p.s_cap = s_cap; p.topk = topk;
+    p.chunk = pl.chunk; p.lay_chunk = pl.lay_chunk; p.per = pl.per;
+    const float scale = sm_scale > 0.f ? sm_scale : 1.0f / sqrtf((float)d);
+    p.qscale = scale * 1.4426950408889634f;
+    p.out_bf16 = out_dt == DS_BF16;
+    p.dense = 0;
+    return launch_decode(kern, p, rows, pl, stream);
+}
+
+ds_status ds_dense_decode(const void* q, const void* k, const void* v, ds_dtype kvdt, int b, int hq,
+                          int hkv, int s, int s_cap, int d, float sm_scale, void* out,
+                          ds_dtype out_dt, cudaStream_t stream) {
+    ds_status r = check_common(b, hq, hkv, s, s_cap, d, kvdt);
+    if (r != DS_OK) return r;
+    if (!q || !k || !v || !out) return fail(DS_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return fail(DS_ERR_INVALID_ARG, "pointer not 16-byte aligned");
+    if (!(out_dt == DS_F32 || (out_dt == DS_BF16 && kvdt == DS_BF16)))
+        return fail(DS_ERR_INVALID_ARG, "out dtype must be DS_F32 or (with bf16 k/v) DS_BF16");
+    const int G = hq / hkv, GT = group_tier(G);
+    const int rows = b * hkv;
+    Plan pl;
+    if (!make_plan(rows, G, s, d, 8, s, true, kCtasPerSm * sm_count(), g_cluster_override.load(), &pl))
+        return fail(DS_ERR_UNSUPPORTED, "no feasible launch plan");
+    ds::DecodeKernel kern = pick_kernel(kvdt, false, d, 8, GT);
+    if (!kern) return fail(DS_ERR_UNSUPPORTED, "no kernel for d=%d G=%d", d, G);
+    ds::DecodeParams p{};
+    p.q = q; p.k = k; p.v = v; p.out = out;
+    p.hkv = hkv; p.G = G; p.s = s; p.s_cap = s_cap; p.topk = s;
+    p.chunk = pl.chunk; p.lay_chunk = 0; p.per = 0;
+    const float scale = sm_scale > 0.f ? sm_scale : 1.0f / sqrtf((float)d);
+    p.qscale = scale * 1.4426950408889634f;
+    p.out_bf16 = out_dt == DS_BF16;
+    p.dense = 1;
+    return launch_decode(kern, p, rows, pl, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,43 @@
+// ds_internal.h -- declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace ds {
+
+struct DecodeParams;
+using DecodeKernel = void (*)(const DecodeParams);
+
+// Kernel instantiation for (k/v dtype, label kind, D, C, GT); nullptr if absent.
+DecodeKernel decode_kernel_f32_fp(int D, int C, int GT);
+DecodeKernel decode_kernel_f32_i4(int D, int C, int GT);
+DecodeKernel decode_kernel_bf16_fp(int D, int C, int GT);
+DecodeKernel decode_kernel_bf16_i4(int D, int C, int GT);
+
+struct LabelArgs {
+    const void* k;
+    bool kdt_bf16;
+    bool int4;
+    const int32_t* idx;
+    int b, hkv, t_begin, t_end, s_cap, d, c;
+    void* label;
+    uint16_t* lscale;
+    uint16_t* lzero;
+};
+cudaError_t launch_label(const LabelArgs& a, cudaStream_t st);
+
+struct CalibArgs {
+    const void* q_win;
+    const void* k;
+    bool bf16;
+    int n, hq, hkv, w, s, d, c;
+    float* ratio;
+    int32_t* idx;
+    void* ws;
+};
+size_t calib_workspace_bytes(int n, int hkv, int d);
+cudaError_t launch_calib(const CalibArgs& a, cudaStream_t st);
+
+}  // namespace ds

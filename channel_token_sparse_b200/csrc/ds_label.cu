@@ -1,0 +1,111 @@
+// ds_label.cu -- label-cache build (prefill) and append (decode) for sm_100a.
+//
+// "大模型稀疏化技术原理：Double Sparsity" (joto.ai), section 离线校准: at prefill
+// every token's heavy key channels are copied from the key cache into the
+// contiguous label cache; at each decode step only the new token's channels
+// are added. The cache may be kept in 4 bits.
+//
+// One CTA handles kTokens consecutive tokens of one (b, kv head) row: the key
+// rows are staged in shared memory with coalesced 16-byte loads, then each
+// label element (fp) or each token (4-bit) is produced from shared memory.
+#include "ds_common.cuh"
+#include "ds_internal.h"
+
+namespace ds {
+
+constexpr int kLabNT = 256;
+constexpr int kTokens = 64;
+
+template <typename TKV, int LK, int D>
+__global__ void __launch_bounds__(kLabNT) ds_label_kernel(const TKV* __restrict__ k,
+                                                          const int32_t* __restrict__ idx, int hkv,
+                                                          int t_begin, int t_end, int s_cap, int c,
+                                                          uint8_t* __restrict__ label,
+                                                          uint16_t* __restrict__ lscale,
+                                                          uint16_t* __restrict__ lzero) {
+    using E = Elem<TKV>;
+    __shared__ __align__(16) TKV rows[kTokens * D];
+    __shared__ int idx_s[128];
+    const int row = blockIdx.y;  // b * hkv + g
+    const int g = row % hkv;
+    const int tb = t_begin + blockIdx.x * kTokens;
+    const int nt = min(kTokens, t_end - tb);
+    if (nt <= 0) return;
+    for (int j = threadIdx.x; j < c; j += kLabNT) idx_s[j] = min(max(idx[(size_t)g * c + j], 0), D - 1);
+
+    const size_t tok0 = (size_t)row * s_cap + tb;
+    constexpr int kVecPerRow = D * E::kBytes / 16;
+    const uint4* src = reinterpret_cast<const uint4*>(k + tok0 * D);
+    uint4* dst = reinterpret_cast<uint4*>(rows);
+    for (int e = threadIdx.x; e < nt * kVecPerRow; e += kLabNT) dst[e] = ldg_stream16(src + e);
+    __syncthreads();
+
+    if constexpr (LK == 0) {
+        TKV* out = reinterpret_cast<TKV*>(label) + tok0 * c;
+        for (int e = threadIdx.x; e < nt * c; e += kLabNT) {
+            const int t = e / c, j = e - t * c;
+            out[e] = rows[t * D + idx_s[j]];
+        }
+    } else {
+        // 4-bit: one thread per token, fp32 arithmetic with IEEE division and
+        // round-half-even, as stated in include/ds.h
+        for (int t = threadIdx.x; t < nt; t += kLabNT) {
+            const TKV* r = rows + t * D;
+            float mn = E::to_f32(r[idx_s[0]]), mx = mn;
+            for (int j = 1; j < c; ++j) {
+                const float x = E::to_f32(r[idx_s[j]]);
+                mn = fminf(mn, x);
+                mx = fmaxf(mx, x);
+            }
+            const float step = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+            const uint16_t sh = __half_as_ushort(__float2half_rn(step));
+            const uint16_t zh = __half_as_ushort(__float2half_rn(mn));
+            const float sc = fp16_bits_to_f32(sh);
+            const float z = fp16_bits_to_f32(zh);
+            uint8_t* o = label + (tok0 + t) * (size_t)(c / 2);
+            for (int j = 0; j < c; j += 2) {
+                uint32_t nib[2];
+#pragma unroll
+                for (int e2 = 0; e2 < 2; ++e2) {
+                    uint32_t code = 0;
+                    if (sc > 0.f) {
+                        float qv = rintf(__fdiv_rn(__fsub_rn(E::to_f32(r[idx_s[j + e2]]), z), sc));
+                        qv = fminf(fmaxf(qv, 0.f), 15.f);
+                        code = (uint32_t)qv;
+                    }
+                    nib[e2] = code;
+                }
+                o[j / 2] = (uint8_t)(nib[0] | (nib[1] << 4));
+            }
+            lscale[tok0 + t] = sh;
+            lzero[tok0 + t] = zh;
+        }
+    }
+}
+
+template <typename TKV, int LK, int D>
+static cudaError_t launch_label_t(const LabelArgs& a, cudaStream_t st) {
+    const int n = a.t_end - a.t_begin;
+    dim3 grid((n + kTokens - 1) / kTokens, a.b * a.hkv);
+    ds_label_kernel<TKV, LK, D><<<grid, kLabNT, 0, st>>>(
+        reinterpret_cast<const TKV*>(a.k), a.idx, a.hkv, a.t_begin, a.t_end, a.s_cap, a.c,
+        reinterpret_cast<uint8_t*>(a.label), a.lscale, a.lzero);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_label(const LabelArgs& a, cudaStream_t st) {
+    const bool i4 = a.int4;
+#define DS_LAB(T, D_)                                                               \
+    if (a.d == D_) return i4 ? launch_label_t<T, 1, D_>(a, st) : launch_label_t<T, 0, D_>(a, st);
+    if (a.kdt_bf16) {
+        DS_LAB(bf16_t, 64)
+        DS_LAB(bf16_t, 128)
+    } else {
+        DS_LAB(float, 64)
+        DS_LAB(float, 128)
+    }
+#undef DS_LAB
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace ds

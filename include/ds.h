@@ -1,0 +1,175 @@
+/*
+ * ds.h -- C ABI of the B200 (sm_100a) Double Sparsity decode-attention library
+ * (libds.so).
+ *
+ * Double Sparsity ("大模型稀疏化技术原理：Double Sparsity", joto.ai blog) speeds up
+ * decode attention in two stages. Offline, a few samples fix the heavy key
+ * channels of each head (section 离线校准). At run time:
+ *   step 1  gather the query's heavy channels,
+ *   step 2  score every cached token approximately against a contiguous "label
+ *           cache" holding only those channels of K (optionally 4-bit),
+ *   step 3  keep the top-k tokens and run exact softmax attention over their
+ *           full K/V rows (section 在线前向计算).
+ * The channel criterion is the importance ratio of "K通道静态性量化方法解析"
+ * (aitangshan.cn) §1.1: r_i = ||Q[i]K[i]^T|| / ||QK^T||.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Pointers are DEVICE pointers owned by the caller, unless stated. The
+ *    library allocates nothing, frees nothing and does not synchronise: work is
+ *    enqueued on `stream` (0 = legacy default stream) and runs asynchronously.
+ *  - Tensors are dense, row-major, with these layouts:
+ *      q        [b, hq, d]                  query of the current decode token
+ *      k, v     [b, hkv, s_cap, d]          key / value cache; tokens [0, s) valid
+ *      idx      [hkv, c]    int32           heavy channels per kv head, each in [0, d)
+ *                                           (kernels clamp out-of-range values into
+ *                                           [0, d); the host does not read idx)
+ *      label    [b, hkv, s_cap, c]          fp label cache (dtype of k), or
+ *               [b, hkv, s_cap, c/2] bytes  4-bit label cache: channel 2j in the
+ *                                           low nibble of byte j, 2j+1 in the high
+ *      lscale, lzero [b, hkv, s_cap]        fp16 bit patterns (4-bit cache only)
+ *      out      [b, hq, d]                  attention output
+ *    Query head h belongs to kv head h / (hq / hkv).
+ *  - Every device pointer must be 16-byte aligned.
+ *  - Arguments are validated before anything is launched. A failed check
+ *    returns DS_ERR_INVALID_ARG (or DS_ERR_UNSUPPORTED for a valid but
+ *    unimplemented shape) and enqueues nothing. A CUDA launch error returns
+ *    DS_ERR_CUDA. ds_last_error() gives a one-line reason for the last
+ *    failure on the calling thread. No exception or exit crosses this ABI.
+ *  - Supported: d in {64, 128}; c in {8, 16, 32, 64, 128} with c <= d;
+ *    hq / hkv <= 8; k/v dtype DS_F32 or DS_BF16; label dtype equal to the k
+ *    dtype or DS_INT4; 1 <= s <= s_cap.
+ */
+#ifndef DS_H
+#define DS_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define DS_API __attribute__((visibility("default")))
+#else
+#define DS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DS_OK = 0,
+    DS_ERR_INVALID_ARG = 1,
+    DS_ERR_UNSUPPORTED = 2,
+    DS_ERR_CUDA = 3,
+    DS_ERR_WORKSPACE = 4
+} ds_status;
+
+typedef enum { DS_F32 = 0, DS_BF16 = 1, DS_F16 = 2, DS_INT4 = 3 } ds_dtype;
+
+/* Human-readable name of a status code (static string). */
+DS_API const char* ds_status_string(ds_status st);
+
+/* One-line reason for the last non-DS_OK status returned on this thread
+ * (static thread-local buffer; empty string if none). */
+DS_API const char* ds_last_error(void);
+
+/* ------------------------------------------------------------ calibration
+ * Offline channel selection ("K通道静态性量化方法解析" §1.1; Double Sparsity
+ * 离线校准). For every calibration sample n and kv head g, Q_g stacks the
+ * observation windows of the group's query heads ((hq/hkv)*w rows) and K_g
+ * holds the s keys:
+ *     r[g, i] = mean_n ||Q_g[:, i] K_g[:, i]^T||_F / ||Q_g K_g^T||_F
+ * (a head with Q_g K_g^T == 0 contributes 0). idx_out[g] receives the c
+ * channels with the largest r (ties to the lower channel), ascending.
+ *
+ *   q_win      [n_samples, hq, w, d]   dtype `dt` (DS_F32 or DS_BF16)
+ *   k          [n_samples, hkv, s, d]  dtype `dt`
+ *   ratio_out  [hkv, d] float32, or NULL
+ *   idx_out    [hkv, c] int32
+ *   ws         caller-owned device scratch of at least
+ *              ds_calibrate_workspace_size() bytes (16-byte aligned); its
+ *              contents on entry do not matter. DS_ERR_WORKSPACE if too small.
+ */
+DS_API ds_status ds_calibrate_workspace_size(int n_samples, int hq, int hkv, int w, int s, int d,
+                                      size_t* bytes);
+DS_API ds_status ds_calibrate_channels(const void* q_win, const void* k, ds_dtype dt,
+                                int n_samples, int hq, int hkv, int w, int s, int d, int c,
+                                float* ratio_out, int32_t* idx_out,
+                                void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* ----------------------------------------------------------- label cache
+ * Prefill (Double Sparsity 离线校准, label cache paragraph): copy the heavy
+ * channels of tokens [0, s) of the key cache into the label cache.
+ *   fp label  : label[b,g,t,j] = k[b,g,t,idx[g,j]]  (bit-exact copy; label_dt == kdt)
+ *   4-bit     : per (b, g, t), in fp32: mn/mx over the c values,
+ *               scale = fp16_rn((mx-mn)/15), zero = fp16_rn(mn),
+ *               code_j = scale > 0 ? clamp(rint((x_j - zero)/scale), 0, 15) : 0
+ *               (IEEE division, round half to even); lscale/lzero receive the
+ *               fp16 bits. Requires c even. Dequantised value: scale*code + zero.
+ * Rows t >= s are not touched.
+ */
+DS_API ds_status ds_build_label_cache(const void* k, ds_dtype kdt, const int32_t* idx,
+                               int b, int hkv, int s, int s_cap, int d, int c,
+                               void* label, ds_dtype label_dt,
+                               uint16_t* lscale, uint16_t* lzero, cudaStream_t stream);
+
+/* Decode-time append: the same copy/pack for the single token at position
+ * `pos` (0 <= pos < s_cap), after the caller has written k[:, :, pos, :]. */
+DS_API ds_status ds_append_label(const void* k, ds_dtype kdt, const int32_t* idx,
+                          int b, int hkv, int pos, int s_cap, int d, int c,
+                          void* label, ds_dtype label_dt,
+                          uint16_t* lscale, uint16_t* lzero, cudaStream_t stream);
+
+/* ------------------------------------------------------ sparse decode step
+ * One decode step of Double Sparsity (在线前向计算 steps 1-3), fused in one
+ * launch. Per batch b and kv head g:
+ *   qL[j]  = sum_{h in group g} q[b, h, idx[g, j]]                  (step 1)
+ *   s_t    = sum_j qL[j] * label[b, g, t, j]        for t < s        (step 2)
+ *            (4-bit: label value scale_t*code + zero_t; fp32 arithmetic)
+ *   sel    = the min(topk, s) tokens with the largest s_t, ties to the
+ *            lower token index (exact on the fp32 scores)             (step 3)
+ *   out[b,h] = softmax_{t in sel}(sm_scale * q[b,h].k[b,g,t]) . v[b,g,t]
+ * topk >= s selects every token (dense attention over the cache).
+ *
+ *   q, k, v    dtype kvdt (DS_F32 or DS_BF16)
+ *   sm_scale   <= 0 selects 1/sqrt(d)
+ *   out        dtype out_dt (DS_F32, or DS_BF16 when kvdt is DS_BF16)
+ *   sel_out    [b, hkv, topk] int32 or NULL: the selected tokens in ascending
+ *              order; entries past min(topk, s) are -1
+ *   score_out  [b, hkv, s] float32 or NULL: the approximate scores s_t
+ * No workspace: scores, the selection and the partial softmax states stay in
+ * on-chip memory of one thread-block cluster per (b, g).
+ */
+DS_API ds_status ds_sparse_decode(const void* q, const void* k, const void* v, ds_dtype kvdt,
+                           const void* label, ds_dtype label_dt,
+                           const uint16_t* lscale, const uint16_t* lzero, const int32_t* idx,
+                           int b, int hq, int hkv, int s, int s_cap, int d, int c, int topk,
+                           float sm_scale, void* out, ds_dtype out_dt,
+                           int32_t* sel_out, float* score_out, cudaStream_t stream);
+
+/* Launch plan of ds_sparse_decode for a shape (host only, launches nothing):
+ * CTAs per thread-block cluster (one cluster per (b, kv head)), tokens per
+ * CTA and dynamic shared memory per CTA in bytes. Any output may be NULL. */
+DS_API ds_status ds_sparse_decode_plan(int b, int hq, int hkv, int s, int d, int c, int topk,
+                                ds_dtype kvdt, ds_dtype label_dt,
+                                int* cluster_out, int* chunk_out, int* smem_out);
+
+/* Force the cluster size (1, 2, 4, 8 or 16 CTAs per (b, kv head) row) used
+ * by ds_sparse_decode, ds_dense_decode and ds_sparse_decode_plan in this
+ * process; 0 restores the automatic choice. A forced size that does not fit
+ * a shape makes those calls return DS_ERR_UNSUPPORTED. Tuning/testing knob. */
+DS_API void ds_sparse_decode_set_cluster(int n);
+
+/* ------------------------------------------------------------- baseline
+ * Dense decode attention over tokens [0, s) of the same cache (no label,
+ * no selection): the measurement baseline the sparse step is compared with.
+ * Same layouts and rules as ds_sparse_decode. */
+DS_API ds_status ds_dense_decode(const void* q, const void* k, const void* v, ds_dtype kvdt,
+                          int b, int hq, int hkv, int s, int s_cap, int d,
+                          float sm_scale, void* out, ds_dtype out_dt, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DS_H */

@@ -214,3 +214,32 @@ def calib_inputs(wl: Workload) -> CalibInputs:
     _plant_q(qw, chans, wl.outlier_scale, wl.g)
     _plant_kv(kc, chans, wl.outlier_scale)
     return CalibInputs(wl, to_storage(qw, wl.kv_dtype), to_storage(kc, wl.kv_dtype), chans)
+
+
+# ------------------------------------------------------------ device inputs
+
+def decode_inputs_torch(wl: Workload, device, s_cap: int | None = None, seed_offset: int = 0):
+    """Same recipe as :func:`decode_inputs`, drawn on ``device`` with torch's
+    seeded generator (for the multi-GB workloads, where drawing on the host is
+    slow). Returns torch tensors (q, k, v) in the workload's dtype; rows past
+    ``wl.s`` are zero. The oracle gets host copies of the rows it checks."""
+    import torch
+
+    s_cap = wl.s if s_cap is None else s_cap
+    dt = torch.float32 if wl.kv_dtype == "f32" else torch.bfloat16
+    gen = torch.Generator(device=device)
+    gen.manual_seed(1000 * wl.index + 100 * seed_offset + 50)
+    chans = torch.from_numpy(outlier_channels(wl)).to(device=device, dtype=torch.long)
+    scale = torch.ones((wl.hkv, wl.d), device=device)
+    scale.scatter_(1, chans, wl.outlier_scale)
+    q = torch.randn((wl.b, wl.hq, wl.d), generator=gen, device=device)
+    q *= scale.repeat_interleave(wl.g, 0)[None]
+    k = torch.zeros((wl.b, wl.hkv, s_cap, wl.d), dtype=dt, device=device)
+    v = torch.zeros((wl.b, wl.hkv, s_cap, wl.d), dtype=dt, device=device)
+    for bb in range(wl.b):  # one batch entry at a time bounds the fp32 temporaries
+        kk = torch.randn((wl.hkv, wl.s, wl.d), generator=gen, device=device)
+        kk *= scale[:, None, :]
+        k[bb, :, : wl.s] = kk.to(dt)
+        v[bb, :, : wl.s] = torch.randn((wl.hkv, wl.s, wl.d), generator=gen, device=device).to(dt)
+        del kk
+    return q.to(dt), k, v
