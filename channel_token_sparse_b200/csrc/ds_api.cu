@@ -8,7 +8,7 @@
 #include <mutex>
 #include <unordered_map>
 
-#include "../../include/ds.h"
+#include "ds.h"
 #include "ds_decode_kernel.cuh"
 #include "ds_internal.h"
 
@@ -60,8 +60,8 @@ int round_up(int x, int m) { return (x + m - 1) / m * m; }
 // grid (rows * N CTAs) still fits in one wave of resident CTAs, keeping at
 // least 256 tokens per CTA; rows beyond one wave use N = 1. A forced N
 // (ds_sparse_decode_set_cluster) overrides the choice when feasible.
-bool make_plan(int rows, int G, int s, int d, int c, int topk, bool dense, int slots, int forced,
-               Plan* out) {
+bool make_plan(int rows, int G, int s, int d, int c, int topk, bool dense, int esz, int slots,
+               int forced, Plan* out) {
     const int GT = group_tier(G);
     const bool select_all = dense || topk >= s;
     const int k_eff = topk < s ? topk : s;
@@ -73,7 +73,7 @@ bool make_plan(int rows, int G, int s, int d, int c, int topk, bool dense, int s
         if (p.chunk > ds::kMaxChunk) continue;
         p.lay_chunk = dense ? 0 : p.chunk;
         p.per = select_all ? 0 : (k_eff + N - 1) / N;
-        p.smem = ds::decode_smem_layout(GT, d, c, p.lay_chunk, p.per).total;
+        p.smem = ds::decode_smem_layout(GT, d, c, p.lay_chunk, p.per, esz).total;
         if (p.smem > kMaxSmem) continue;
         if (forced) {
             if (N == forced) { *out = p; return true; }
@@ -243,7 +243,8 @@ ds_status ds_sparse_decode_plan(int b, int hq, int hkv, int s, int d, int c, int
     if (label_dt != DS_INT4 && label_dt != kvdt) return fail(DS_ERR_INVALID_ARG, "label dtype");
     if (topk < 1) return fail(DS_ERR_INVALID_ARG, "topk must be >= 1");
     Plan pl;
-    if (!make_plan(b * hkv, hq / hkv, s, d, c, topk, false, kCtasPerSm * 148, g_cluster_override.load(), &pl))
+    if (!make_plan(b * hkv, hq / hkv, s, d, c, topk, false, kvdt == DS_F32 ? 4 : 2, kCtasPerSm * 148,
+                   g_cluster_override.load(), &pl))
         return fail(DS_ERR_UNSUPPORTED, "no feasible launch plan (s too long for 16 CTAs per row)");
     if (cluster_out) *cluster_out = pl.N;
     if (chunk_out) *chunk_out = pl.chunk;
@@ -270,7 +271,8 @@ ds_status ds_sparse_decode(const void* q, const void* k, const void* v, ds_dtype
     const int G = hq / hkv, GT = group_tier(G);
     const int rows = b * hkv;
     Plan pl;
-    if (!make_plan(rows, G, s, d, c, topk, false, kCtasPerSm * sm_count(), g_cluster_override.load(), &pl))
+    if (!make_plan(rows, G, s, d, c, topk, false, kvdt == DS_F32 ? 4 : 2, kCtasPerSm * sm_count(),
+                   g_cluster_override.load(), &pl))
         return fail(DS_ERR_UNSUPPORTED, "no feasible launch plan (s too long for 16 CTAs per row)");
     ds::DecodeKernel kern = pick_kernel(kvdt, label_dt == DS_INT4, d, c, GT);
     if (!kern) return fail(DS_ERR_UNSUPPORTED, "no kernel for d=%d c=%d G=%d", d, c, G);
@@ -299,7 +301,8 @@ ds_status ds_dense_decode(const void* q, const void* k, const void* v, ds_dtype 
     const int G = hq / hkv, GT = group_tier(G);
     const int rows = b * hkv;
     Plan pl;
-    if (!make_plan(rows, G, s, d, 8, s, true, kCtasPerSm * sm_count(), g_cluster_override.load(), &pl))
+    if (!make_plan(rows, G, s, d, 8, s, true, kvdt == DS_F32 ? 4 : 2, kCtasPerSm * sm_count(),
+                   g_cluster_override.load(), &pl))
         return fail(DS_ERR_UNSUPPORTED, "no feasible launch plan");
     ds::DecodeKernel kern = pick_kernel(kvdt, false, d, 8, GT);
     if (!kern) return fail(DS_ERR_UNSUPPORTED, "no kernel for d=%d G=%d", d, G);

@@ -81,6 +81,53 @@ __device__ __forceinline__ void load_words(uint32_t (&w)[N / 4], const uint8_t* 
     }
 }
 
+// Shared-memory loads of N bytes (N in {4, 8, 16}) into N/4 registers.
+template <int N>
+__device__ __forceinline__ void lds_words(uint32_t (&w)[N / 4], const uint8_t* p) {
+    if constexpr (N == 16) {
+        const uint4 x = *reinterpret_cast<const uint4*>(p);
+        w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
+    } else if constexpr (N == 8) {
+        const uint2 x = *reinterpret_cast<const uint2*>(p);
+        w[0] = x.x; w[1] = x.y;
+    } else {
+        static_assert(N == 4, "lds size");
+        w[0] = *reinterpret_cast<const uint32_t*>(p);
+    }
+}
+
+// 16-byte asynchronous global -> shared copy (LDGSTS, L2 only), and its
+// group bookkeeping. Completion is awaited per thread with cp_async_wait;
+// other lanes' copies become visible after a __syncwarp / __syncthreads.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Bulk prefetch of [p, p + bytes) into L2 (TMA unit; no registers held while
+// in flight). p must be 16-byte aligned and bytes a multiple of 16.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Prefetch the byte range [base + lo, base + hi) in pieces of `piece` bytes
+// (a multiple of 16), one piece per thread index `who`. The range is trimmed
+// inward to 16-byte aligned ABSOLUTE addresses (row bases of small-row arrays,
+// e.g. fp16 scales at row * s_cap * 2 bytes, need not be aligned), so every
+// prefetch starts on a 16-byte boundary and covers a multiple of 16 bytes.
+__device__ __forceinline__ void prefetch_range(const uint8_t* base, size_t lo, size_t hi, int who,
+                                               uint32_t piece) {
+    const uintptr_t a = (reinterpret_cast<uintptr_t>(base + lo) + 15) & ~(uintptr_t)15;
+    const uintptr_t e = reinterpret_cast<uintptr_t>(base + hi) & ~(uintptr_t)15;
+    const uintptr_t start = a + (uintptr_t)who * piece;
+    if (start >= e) return;
+    const uintptr_t n = e - start < piece ? e - start : piece;
+    prefetch_l2(reinterpret_cast<const void*>(start), (uint32_t)n);
+}
+
 // Order-preserving map of an fp32 score to uint32: larger score -> larger key.
 // -0 is folded onto +0 so that equal scores give equal keys.
 __device__ __forceinline__ uint32_t score_key(float s) {

@@ -37,6 +37,8 @@ constexpr int kNW = kNT / 32;        // warps per CTA
 constexpr int kMaxChunk = 32768;     // tokens per CTA (16-bit keys -> 64 KiB)
 constexpr int kLabelInt4 = 1;
 constexpr int kLabelFp = 0;
+constexpr uint32_t kPfPiece = 4096;  // bytes per L2 bulk-prefetch instruction
+constexpr int kPfRounds = 2;         // scoring rounds prefetched ahead
 
 struct DecodeParams {
     const void* q;
@@ -60,12 +62,28 @@ struct DecodeParams {
 
 // Shared-memory carve-up (bytes), identical on host and device.
 struct DecodeSmem {
-    int qs, qL, idx, histA, histB, ctl, scan, cm, cl, co, bits, sel, region, total;
+    int qs, qL, idx, histA, histB, ctl, scan, cm, cl, co, bits, blist, sel, region, total;
 };
 
 __host__ __device__ inline int align16(int x) { return (x + 15) & ~15; }
 
-__host__ __device__ inline DecodeSmem decode_smem_layout(int GT, int D, int C, int chunk, int per) {
+// Attention-phase staging: each warp owns a ring of kAttStages stages; a
+// stage holds the K rows then the V rows of att_stage_tokens(row bytes)
+// tokens (~2 KiB per stage). A warp's partial softmax state (at most
+// 8 * (128 + 2) floats) is later written into its own ring.
+constexpr int kAttStages = 4;
+// Tokens of the k-th key's 16-bit bucket kept in a list for the last radix
+// pass (a CTA whose bucket is larger falls back to sweeping its keys).
+constexpr int kBucketCap = 1024;
+__host__ __device__ constexpr int att_stage_tokens(int row_bytes) {
+    return row_bytes >= 1024 ? 1 : 1024 / row_bytes;
+}
+__host__ __device__ constexpr int att_ring_bytes(int row_bytes) {
+    return kAttStages * att_stage_tokens(row_bytes) * 2 * row_bytes;
+}
+
+__host__ __device__ inline DecodeSmem decode_smem_layout(int GT, int D, int C, int chunk, int per,
+                                                         int elem_bytes) {
     DecodeSmem L;
     int o = 0;
     L.qs = o;     o += align16(GT * D * 4);
@@ -78,18 +96,19 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int GT, int D, int C, i
     L.cm = o;     o += align16(GT * 4);
     L.cl = o;     o += align16(GT * 4);
     L.co = o;     o += align16(GT * D * 4);
-    L.bits = o;   o += align16((chunk / 32) * 4);
+    L.bits = o;   o += align16(chunk / 8);
+    L.blist = o;  o += chunk > 0 ? kBucketCap * 4 : 0;
     L.sel = o;    o += align16(per * 4);
     L.region = o;
     const int keys = chunk * 2;
-    const int parts = kNW * GT * (D + 2) * 4;
-    o += align16(keys > parts ? keys : parts);
+    const int ring = kNW * att_ring_bytes(D * elem_bytes);
+    o += align16(keys > ring ? keys : ring);
     L.total = o;
     return L;
 }
 
 // ctl[] slots
-enum { kCtlBin = 0, kCtlNeed = 1, kCtlCnt = 2, kCtlCS = 4, kCtlCT = 5, kCtlP = 6, kCtlTP = 7 };
+enum { kCtlBin = 0, kCtlNeed = 1, kCtlCnt = 2, kCtlCS = 4, kCtlCT = 5, kCtlP = 6, kCtlTP = 7, kCtlBL = 8 };
 
 // Row geometry of the label cache.
 template <typename TKV, int LK, int C>
@@ -137,25 +156,21 @@ __device__ __forceinline__ float label_score(const uint32_t (&w)[LabelGeom<TKV, 
     }
 }
 
-// Warp-aggregated histogram increment; bin >= 256 means "no count". Must be
-// called by all 32 lanes.
-__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin) {
-    const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-    const int leader = __ffs(peers) - 1;
-    if (lane_id() == leader && bin < 256u) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
-}
-
 // Sum a 256-bin histogram over the cluster (DSMEM) and find the bin holding
 // the `need`-th largest key. Writes ctl[kCtlBin], ctl[kCtlNeed] (how many to
 // take from that bin) and ctl[kCtlCnt] (the bin's size). Requires a cluster
 // barrier before (histograms complete); ends with __syncthreads().
+// `zero_next` (may be null) is the other histogram buffer: no CTA reads it
+// any more once every CTA has passed the barrier before this call, so it is
+// cleared here for the next pass.
 __device__ __forceinline__ void cluster_select_bin(cg::cluster_group& cluster, uint32_t* hist,
                                                    int nblocks, uint32_t need, int* ctl,
-                                                   uint32_t* scan) {
+                                                   uint32_t* scan, uint32_t* zero_next) {
     const int tid = threadIdx.x;
     const int bin = 255 - tid;  // thread 0 holds the largest bin
     uint32_t cnt = 0;
     for (int r = 0; r < nblocks; ++r) cnt += cluster.map_shared_rank(hist, r)[bin];
+    if (zero_next) zero_next[tid] = 0u;
     uint32_t total;
     const uint32_t excl = block_excl_scan<kNT>(cnt, scan, &total);
     if (excl < need && need <= excl + cnt) {
@@ -172,10 +187,6 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     using LG = LabelGeom<TKV, LK, C>;
     constexpr int EPL = D / 32;                       // elements of a K/V row per lane
     constexpr int RBL = EPL * E::kBytes;              // bytes of a K/V row per lane
-    // tokens per warp batch: ~64 B of K plus 64 B of V in flight per lane,
-    // fewer when several query heads share the kv head (registers)
-    constexpr int TB0 = (64 / RBL) < 4 ? 4 : ((64 / RBL) > 8 ? 8 : (64 / RBL));
-    constexpr int TB = GT >= 8 ? (TB0 / 4 < 2 ? 2 : TB0 / 4) : GT >= 4 ? (TB0 / 2 < 2 ? 2 : TB0 / 2) : TB0;
     static_assert(EPL * 32 == D, "D must be a multiple of 32");
 
     cg::cluster_group cluster = cg::this_cluster();
@@ -187,7 +198,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     const int tid = threadIdx.x, lane = lane_id(), wid = warp_id();
 
     extern __shared__ __align__(16) uint8_t smem[];
-    const DecodeSmem L = decode_smem_layout(GT, D, C, p.lay_chunk, p.per);
+    const DecodeSmem L = decode_smem_layout(GT, D, C, p.lay_chunk, p.per, E::kBytes);
     float* qs = reinterpret_cast<float*>(smem + L.qs);
     float* qLs = reinterpret_cast<float*>(smem + L.qL);
     int* idx_s = reinterpret_cast<int*>(smem + L.idx);
@@ -198,10 +209,10 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     float* cm = reinterpret_cast<float*>(smem + L.cm);
     float* cl = reinterpret_cast<float*>(smem + L.cl);
     float* co = reinterpret_cast<float*>(smem + L.co);
-    uint32_t* bits = reinterpret_cast<uint32_t*>(smem + L.bits);
+    uint8_t* bits8 = smem + L.bits;                     // bucket flags, one byte per 8 tokens
+    uint32_t* blist = reinterpret_cast<uint32_t*>(smem + L.blist);
     int* sel_list = reinterpret_cast<int*>(smem + L.sel);
     uint16_t* keys = reinterpret_cast<uint16_t*>(smem + L.region);
-    float* wpart = reinterpret_cast<float*>(smem + L.region);  // after compaction
 
     const int s = p.s;
     const int t0 = rank * p.chunk;
@@ -211,14 +222,36 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     const int k_eff = min(p.topk, s);
     const bool select_all = p.dense || p.topk >= s;
 
+    // [phase] 0
+    const uint8_t* lab = reinterpret_cast<const uint8_t*>(p.label) + row_tok * LG::kBytes;
+    const uint16_t* lsc = (LK == kLabelInt4) ? p.lscale + row_tok : nullptr;
+    const uint16_t* lze = (LK == kLabelInt4) ? p.lzero + row_tok : nullptr;
+    const bool need_scores = !p.dense && (!select_all || p.score_out != nullptr);
+    constexpr int U = LG::kU;
+    constexpr int kRound = kNT * U;  // tokens per scoring round
+    // Start pulling the first rounds of this CTA's label rows into L2 while
+    // the query is set up; the scoring loop keeps kPfRounds rounds ahead.
+    auto prefetch_label_round = [&](int r) {
+        const size_t lo = (size_t)(t0 + r * kRound), hi = (size_t)(t0 + min(n_loc, (r + 1) * kRound));
+        if (r * kRound >= n_loc) return;
+        constexpr int kPieces = (kRound * LG::kBytes + kPfPiece - 1) / kPfPiece;
+        if (tid < kPieces) prefetch_range(lab, lo * LG::kBytes, hi * LG::kBytes, tid, kPfPiece);
+        if constexpr (LK == kLabelInt4) {
+            if (tid == kPieces) prefetch_range(reinterpret_cast<const uint8_t*>(lsc), lo * 2, hi * 2, 0, kRound * 2);
+            if (tid == kPieces + 1) prefetch_range(reinterpret_cast<const uint8_t*>(lze), lo * 2, hi * 2, 0, kRound * 2);
+        }
+    };
+
     // ---------------------------------------------------------- setup, step 1
     for (int e = tid; e < G * D; e += kNT) qs[e] = E::to_f32(qrow[e]);
     if (!p.dense) {
         for (int j = tid; j < C; j += kNT) idx_s[j] = min(max(p.idx[(size_t)g * C + j], 0), D - 1);
         histA[tid] = 0u;
         histB[tid] = 0u;
-        for (int e = tid; e < p.lay_chunk / 32; e += kNT) bits[e] = 0u;
+        if (tid == 0) ctl[kCtlBL] = 0;
     }
+    if (need_scores)  // after the q / idx loads, so they do not queue behind it
+        for (int r = 0; r <= kPfRounds; ++r) prefetch_label_round(r);
     __syncthreads();
     if (!p.dense) {
         for (int j = tid; j < C; j += kNT) {
@@ -229,9 +262,6 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     }
     __syncthreads();
 
-    const uint8_t* lab = reinterpret_cast<const uint8_t*>(p.label) + row_tok * LG::kBytes;
-    const uint16_t* lsc = (LK == kLabelInt4) ? p.lscale + row_tok : nullptr;
-    const uint16_t* lze = (LK == kLabelInt4) ? p.lzero + row_tok : nullptr;
     float qreg[C <= 32 ? C : 1];
     float qsum = 0.f;
 
@@ -248,7 +278,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         return label_score<TKV, LK, C>(w, qreg, qLs, sc, z, qsum);
     };
 
-    if (!select_all) {
+    if (need_scores) {
         if constexpr (C <= 32) {
 #pragma unroll
             for (int j = 0; j < C; ++j) qreg[j] = qLs[j];
@@ -256,10 +286,11 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         for (int j = 0; j < C; ++j) qsum += qLs[j];
     }
 
+    // [phase] 1
     // ---------------------------------------------------------------- step 2
-    if (!p.dense && (!select_all || p.score_out != nullptr)) {
-        constexpr int U = LG::kU;
-        for (int base = 0; base < n_loc; base += kNT * U) {
+    if (need_scores) {
+        for (int base = 0; base < n_loc; base += kRound) {
+            prefetch_label_round(base / kRound + kPfRounds + 1);
             uint32_t w[U][LG::kWords];
             float sc[U], z[U];
 #pragma unroll
@@ -289,92 +320,147 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
                     }
                     if (p.score_out) p.score_out[(size_t)row * s + t0 + i] = sv;
                 }
-                if (!select_all) hist_add(histA, bin);
+                if (!select_all && bin < 256u) atomicAdd(&histA[bin], 1u);
             }
         }
     }
 
+    // [phase] 2
     // --------------------------------------------------------------- step 3a
     int T16 = 0, Tlo = 0, r_tie = 0;
     bool refine = false;
     if (!select_all) {
         cluster.sync();                                        // histograms A complete
-        cluster_select_bin(cluster, histA, N, (uint32_t)k_eff, ctl, scan);
+        cluster_select_bin(cluster, histA, N, (uint32_t)k_eff, ctl, scan, nullptr);
         const int bA = ctl[kCtlBin];
         const int needA = ctl[kCtlNeed];
-        for (int base = 0; base < n_loc; base += kNT) {
-            const int i = base + tid;
-            uint32_t bin = 256u;
-            if (i < n_loc) {
-                const uint32_t k16 = keys[i];
-                if ((int)(k16 >> 8) == bA) bin = k16 & 255u;
+        // [phase] 3
+        // Key sweeps read 8 keys (16 bytes) per thread per step; group g holds
+        // local tokens [8g, 8g + 8). Keys past n_loc in the last group are masked.
+        const uint8_t* kbytes = reinterpret_cast<const uint8_t*>(keys);
+        const int ngrp = (n_loc + 7) >> 3;
+        auto key8 = [&](int grp, uint32_t (&w)[4]) { lds_words<16>(w, kbytes + grp * 16); };
+        auto kat = [](const uint32_t (&w)[4], int e) -> int { return (int)((w[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu); };
+        for (int grp = tid; grp < ngrp; grp += kNT) {
+            uint32_t w[4];
+            key8(grp, w);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int k16 = kat(w, e);
+                if (grp * 8 + e < n_loc && (k16 >> 8) == bA) atomicAdd(&histB[k16 & 255], 1u);
             }
-            hist_add(histB, bin);
         }
+        // [phase] 10
         cluster.sync();                                        // histograms B complete
-        cluster_select_bin(cluster, histB, N, (uint32_t)needA, ctl, scan);
+        // [phase] 11
+        cluster_select_bin(cluster, histB, N, (uint32_t)needA, ctl, scan, histA);
         T16 = (bA << 8) | ctl[kCtlBin];
         const int needB = ctl[kCtlNeed];
         refine = needB < ctl[kCtlCnt];
+        // [phase] 4
         if (refine) {
-            // the k-th key's 16-bit bucket is split: re-score its tokens exactly
-            histA[tid] = 0u;
-            __syncthreads();
-            for (int base = 0; base < n_loc; base += kNT) {
-                const int i = base + tid;
-                bool inb = false;
-                uint32_t bin = 256u;
-                if (i < n_loc && (int)keys[i] == T16) {
-                    inb = true;
+            // The k-th key's 16-bit bucket is split: re-score its tokens
+            // (bit-identical arithmetic), keep their low 16 key bits in place
+            // of the high ones, flag them, and list them for pass D.
+            for (int grp = tid; grp < ngrp; grp += kNT) {
+                uint32_t w[4];
+                key8(grp, w);
+                uint32_t flags = 0;
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if (grp * 8 + e < n_loc && kat(w, e) == T16) flags |= 1u << e;
+                bits8[grp] = (uint8_t)flags;
+                for (uint32_t m = flags; m; m &= m - 1) {
+                    const int i = grp * 8 + __ffs(m) - 1;
                     const uint32_t low = score_key(rescore(t0 + i)) & 0xFFFFu;
                     keys[i] = (uint16_t)low;
-                    bin = low >> 8;
+                    atomicAdd(&histA[low >> 8], 1u);
+                    const int slot = atomicAdd(&ctl[kCtlBL], 1);
+                    if (slot < kBucketCap) blist[slot] = low | ((uint32_t)i << 16);
                 }
-                const uint32_t m = __ballot_sync(0xffffffffu, inb);
-                if (lane == 0 && (base + wid * 32) < n_loc) bits[(base + wid * 32) >> 5] = m;
-                hist_add(histA, bin);
             }
+            // [phase] 12
             cluster.sync();                                    // histograms C complete
-            cluster_select_bin(cluster, histA, N, (uint32_t)needB, ctl, scan);
+            // [phase] 13
+            cluster_select_bin(cluster, histA, N, (uint32_t)needB, ctl, scan, histB);
             const int bC = ctl[kCtlBin];
             const int needC = ctl[kCtlNeed];
-            histB[tid] = 0u;
-            __syncthreads();
-            for (int base = 0; base < n_loc; base += kNT) {
-                const int i = base + tid;
-                uint32_t bin = 256u;
-                if (i < n_loc && ((bits[i >> 5] >> (i & 31)) & 1u)) {
-                    const uint32_t low = keys[i];
-                    if ((int)(low >> 8) == bC) bin = low & 255u;
+            const int nbl = ctl[kCtlBL];
+            if (nbl <= kBucketCap) {
+                for (int j = tid; j < nbl; j += kNT) {
+                    const uint32_t low = blist[j] & 0xFFFFu;
+                    if ((int)(low >> 8) == bC) atomicAdd(&histB[low & 255u], 1u);
                 }
-                hist_add(histB, bin);
+            } else {
+                for (int grp = tid; grp < ngrp; grp += kNT) {
+                    const uint32_t fl = bits8[grp];
+                    if (!fl) continue;
+                    uint32_t w[4];
+                    key8(grp, w);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int low = kat(w, e);
+                        if (((fl >> e) & 1u) && (low >> 8) == bC) atomicAdd(&histB[low & 255], 1u);
+                    }
+                }
             }
+            // [phase] 14
             cluster.sync();                                    // histograms D complete
-            cluster_select_bin(cluster, histB, N, (uint32_t)needC, ctl, scan);
+            // [phase] 15
+            cluster_select_bin(cluster, histB, N, (uint32_t)needC, ctl, scan, nullptr);
             Tlo = (bC << 8) | ctl[kCtlBin];
             r_tie = ctl[kCtlNeed];
         }
 
+        // [phase] 5
         // ----------------------------------------------------- compaction
-        // classes: 1 = selected outright, 2 = exact tie with the k-th key
-        const int run = (n_loc + kNT - 1) / kNT;
-        const int i0 = min(n_loc, tid * run), i1 = min(n_loc, i0 + run);
-        auto klass = [&](int i) -> int {
-            const int k16 = keys[i];
+        // classes: 1 = selected outright, 2 = exact tie with the k-th key.
+        // Warp w owns a contiguous segment of key groups; in each step lane l
+        // reads group seg + 32*step + l (conflict-free 16-byte loads), so lane
+        // order is index order and warp scans rank the selected tokens.
+        auto klass = [&](int k16, bool inb) -> int {
             if (!refine) return k16 >= T16 ? 1 : 0;
-            if ((bits[i >> 5] >> (i & 31)) & 1u) return k16 > Tlo ? 1 : (k16 == Tlo ? 2 : 0);
+            if (inb) return k16 > Tlo ? 1 : (k16 == Tlo ? 2 : 0);
             return k16 > T16 ? 1 : 0;
         };
+        // per group: strict count in bits 0..7, tie count in bits 8..15, and
+        // the class of each of its 8 keys (2 bits each) in bits 16..31
+        auto classify8 = [&](int grp) -> uint32_t {
+            if (grp >= ngrp) return 0u;
+            uint32_t w[4];
+            key8(grp, w);
+            const uint32_t fl = refine ? bits8[grp] : 0u;
+            uint32_t r = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const uint32_t c = grp * 8 + e < n_loc ? (uint32_t)klass(kat(w, e), (fl >> e) & 1u) : 0u;
+                r += (c == 1u) + ((c == 2u) << 8) + (c << (16 + 2 * e));
+            }
+            return r;
+        };
+        const int gpw = (((ngrp + kNW - 1) / kNW) + 31) & ~31;   // groups per warp
+        const int wg0 = wid * gpw, wg1 = min(ngrp, wg0 + gpw);
         uint32_t ns = 0, nt = 0;
-        for (int i = i0; i < i1; ++i) {
-            const int c = klass(i);
-            ns += c == 1;
-            nt += c == 2;
+        for (int grp = wg0 + lane; grp - lane < wg1; grp += 32) {
+            const uint32_t r = grp < wg1 ? classify8(grp) : 0u;
+            ns += r & 255u;
+            nt += (r >> 8) & 255u;
         }
-        uint32_t tot;
-        const uint32_t ex = block_excl_scan<kNT>((ns << 16) | nt, scan, &tot);
-        if (tid == 0) { ctl[kCtlCS] = (int)(tot >> 16); ctl[kCtlCT] = (int)(tot & 0xFFFFu); }
+        ns = (uint32_t)__reduce_add_sync(0xffffffffu, ns);
+        nt = (uint32_t)__reduce_add_sync(0xffffffffu, nt);
+        if (lane == 0) scan[wid] = (ns << 16) | nt;
+        __syncthreads();
+        if (wid == 0) {
+            const uint32_t x = lane < kNW ? scan[lane] : 0u;
+            const uint32_t xi = warp_incl_scan(x);
+            __syncwarp();
+            if (lane < kNW) scan[lane] = xi - x;
+            if (lane == kNW - 1) { ctl[kCtlCS] = (int)(xi >> 16); ctl[kCtlCT] = (int)(xi & 0xFFFFu); }
+        }
+        // [phase] 16
+        // [phase] 17
         cluster.sync();                                        // per-CTA counts visible
+        // [phase] 18
         if (wid == 0) {
             int cs = 0, ct = 0;
             if (lane < N) {
@@ -390,23 +476,35 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
             if (lane == rank) { ctl[kCtlP] = p_incl - cnt; ctl[kCtlTP] = tp; }
         }
         __syncthreads();
+        // [phase] 19
         const int P = ctl[kCtlP], TP = ctl[kCtlTP];
-        const int ex_s = (int)(ex >> 16), ex_t = (int)(ex & 0xFFFFu);
-        int pos = P + ex_s + (refine ? max(0, min(ex_t, r_tie - TP)) : 0);
-        int tie_rank = TP + ex_t;
+        const int tie_quota = max(0, r_tie - TP);  // ties this CTA may still take
+        int sb = (int)(scan[wid] >> 16), tb = (int)(scan[wid] & 0xFFFFu);  // before this step
         const int per = p.per;
-        for (int i = i0; i < i1; ++i) {
-            const int c = klass(i);
-            bool take = c == 1;
-            if (c == 2) { take = tie_rank < r_tie; ++tie_rank; }
-            if (take) {
-                const int dst = pos / per;
-                int* rl = cluster.map_shared_rank(sel_list, dst);
-                rl[pos - dst * per] = t0 + i;
-                if (p.sel_out) p.sel_out[(size_t)row * p.topk + pos] = t0 + i;
-                ++pos;
+        for (int grp = wg0 + lane; grp - lane < wg1; grp += 32) {
+            const uint32_t r = grp < wg1 ? classify8(grp) : 0u;
+            const uint32_t cs_l = r & 255u, ct_l = (r >> 8) & 255u;
+            const uint32_t pk = (cs_l << 16) | ct_l;
+            const uint32_t incl = warp_incl_scan(pk);
+            int my_sb = sb + (int)((incl - pk) >> 16), my_tb = tb + (int)((incl - pk) & 0xFFFFu);
+            const uint32_t tot_step = __shfl_sync(0xffffffffu, incl, 31);
+            sb += (int)(tot_step >> 16);
+            tb += (int)(tot_step & 0xFFFFu);
+            for (uint32_t cls = r >> 16, e = 0; cls; cls >>= 2, ++e) {
+                const uint32_t c = cls & 3u;
+                if (c == 1u || (c == 2u && my_tb < tie_quota)) {
+                    const int pos = P + my_sb + min(my_tb, tie_quota);
+                    const int dst = pos / per;
+                    int* rl = cluster.map_shared_rank(sel_list, dst);
+                    const int t = t0 + grp * 8 + (int)e;
+                    rl[pos - dst * per] = t;
+                    if (p.sel_out) p.sel_out[(size_t)row * p.topk + pos] = t;
+                }
+                my_sb += c == 1u;
+                my_tb += c == 2u;
             }
         }
+        // [phase] 20
         cluster.sync();                                        // selection lists complete
     } else if (p.sel_out) {
         for (int i = tid; i < n_loc; i += kNT) p.sel_out[(size_t)row * p.topk + t0 + i] = t0 + i;
@@ -414,10 +512,38 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
             for (int j = s + tid; j < p.topk; j += kNT) p.sel_out[(size_t)row * p.topk + j] = -1;
     }
 
+    // [phase] 6
     // --------------------------------------------------------------- step 3b
-    const int n_att = select_all ? n_loc : max(0, min(p.per, k_eff - rank * p.per));
+    // Each warp streams the K and V rows of its tokens through a ring of
+    // kAttStages shared-memory stages with cp.async (16-byte LDGSTS, no
+    // registers held while in flight), kAttStages-1 stages ahead of compute.
     const TKV* kb = reinterpret_cast<const TKV*>(p.k) + row_tok * D;
     const TKV* vb = reinterpret_cast<const TKV*>(p.v) + row_tok * D;
+    constexpr int RB = D * E::kBytes;              // bytes of one K or V row
+    constexpr int TBS = att_stage_tokens(RB);      // tokens per stage
+    constexpr int kStageBytes = 2 * TBS * RB;
+    constexpr int kPiecesPerRow = RB / 16;
+    const int n_att = select_all ? n_loc : max(0, min(p.per, k_eff - rank * p.per));
+    uint8_t* ring = smem + L.region + wid * att_ring_bytes(RB);
+    const int nb = n_att > wid * TBS ? (n_att - wid * TBS + kNW * TBS - 1) / (kNW * TBS) : 0;
+    auto att_token = [&](int j) -> int { return select_all ? t0 + j : sel_list[j]; };
+    auto issue_stage = [&](int bi) {
+        const int bt0 = (wid + bi * kNW) * TBS;
+        uint8_t* st = ring + (bi % kAttStages) * kStageBytes;
+        for (int pc = lane; pc < 2 * TBS * kPiecesPerRow; pc += 32) {
+            const int r = pc / kPiecesPerRow, off = (pc - r * kPiecesPerRow) * 16;
+            const int u = r < TBS ? r : r - TBS;
+            if (bt0 + u < n_att) {
+                const TKV* src = (r < TBS ? kb : vb) + (size_t)att_token(bt0 + u) * D;
+                cp_async16(st + r * RB + off, reinterpret_cast<const uint8_t*>(src) + off);
+            }
+        }
+    };
+#pragma unroll 1
+    for (int bi = 0; bi < kAttStages - 1; ++bi) {
+        if (bi < nb) issue_stage(bi);
+        cp_async_commit();
+    }
 
     float qf[GT][EPL];
 #pragma unroll
@@ -435,30 +561,27 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         for (int e = 0; e < EPL; ++e) o_run[h][e] = 0.f;
     }
 
-    for (int bt = wid * TB; bt < n_att; bt += kNW * TB) {
-        uint32_t kw[TB][RBL / 4 > 0 ? RBL / 4 : 1], vw[TB][RBL / 4 > 0 ? RBL / 4 : 1];
-        bool ok[TB];
+    // [phase] 21
+#pragma unroll 1
+    for (int bi = 0; bi < nb; ++bi) {
+        if (bi + kAttStages - 1 < nb) issue_stage(bi + kAttStages - 1);
+        cp_async_commit();
+        cp_async_wait<kAttStages - 1>();
+        __syncwarp();
+        const uint8_t* st = ring + (bi % kAttStages) * kStageBytes;
+        const int bt0 = (wid + bi * kNW) * TBS;
+        bool ok[TBS];
+        float zt[TBS][GT];
 #pragma unroll
-        for (int u = 0; u < TB; ++u) {
-            const int j = bt + u;
-            ok[u] = j < n_att;
-            if (ok[u]) {
-                const int t = select_all ? t0 + j : sel_list[j];
-                load_words<RBL>(kw[u], reinterpret_cast<const uint8_t*>(kb + (size_t)t * D + lane * EPL));
-                load_words<RBL>(vw[u], reinterpret_cast<const uint8_t*>(vb + (size_t)t * D + lane * EPL));
-            } else {
-#pragma unroll
-                for (int e = 0; e < RBL / 4; ++e) { kw[u][e] = 0u; vw[u][e] = 0u; }
-            }
-        }
-        float zt[TB][GT];
-#pragma unroll
-        for (int u = 0; u < TB; ++u) {
+        for (int u = 0; u < TBS; ++u) {
+            ok[u] = bt0 + u < n_att;
+            uint32_t kw[RBL / 4 > 0 ? RBL / 4 : 1];
+            lds_words<RBL>(kw, st + u * RB + lane * RBL);
             float kf[EPL];
 #pragma unroll
             for (int e = 0; e < EPL; ++e) {
-                if constexpr (E::kBytes == 2) kf[e] = (e & 1) ? bf16hi(kw[u][e >> 1]) : bf16lo(kw[u][e >> 1]);
-                else kf[e] = __uint_as_float(kw[u][e]);
+                if constexpr (E::kBytes == 2) kf[e] = (e & 1) ? bf16hi(kw[e >> 1]) : bf16lo(kw[e >> 1]);
+                else kf[e] = __uint_as_float(kw[e]);
             }
 #pragma unroll
             for (int h = 0; h < GT; ++h) {
@@ -473,33 +596,39 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
             if (h >= G) break;
             float mx = -INFINITY;
 #pragma unroll
-            for (int u = 0; u < TB; ++u) if (ok[u]) mx = fmaxf(mx, zt[u][h]);
+            for (int u = 0; u < TBS; ++u) if (ok[u]) mx = fmaxf(mx, zt[u][h]);
             const float m_new = fmaxf(m_run[h], mx);
             const float corr = exp2f(m_run[h] - m_new);
             float l = l_run[h] * corr;
 #pragma unroll
             for (int e = 0; e < EPL; ++e) o_run[h][e] *= corr;
 #pragma unroll
-            for (int u = 0; u < TB; ++u) {
+            for (int u = 0; u < TBS; ++u) {
                 if (!ok[u]) continue;
                 const float pr = exp2f(zt[u][h] - m_new);
                 l += pr;
+                uint32_t vw[RBL / 4 > 0 ? RBL / 4 : 1];
+                lds_words<RBL>(vw, st + (TBS + u) * RB + lane * RBL);
 #pragma unroll
                 for (int e = 0; e < EPL; ++e) {
                     float vf;
-                    if constexpr (E::kBytes == 2) vf = (e & 1) ? bf16hi(vw[u][e >> 1]) : bf16lo(vw[u][e >> 1]);
-                    else vf = __uint_as_float(vw[u][e]);
+                    if constexpr (E::kBytes == 2) vf = (e & 1) ? bf16hi(vw[e >> 1]) : bf16lo(vw[e >> 1]);
+                    else vf = __uint_as_float(vw[e]);
                     o_run[h][e] = fmaf(pr, vf, o_run[h][e]);
                 }
             }
             m_run[h] = m_new;
             l_run[h] = l;
         }
+        __syncwarp();
     }
+    cp_async_wait<0>();
+    __syncwarp();
 
-    // per-warp partials -> shared memory (the key region is free now)
+    // [phase] 7
+    // per-warp partials -> the warp's own ring (its copies have all landed)
     {
-        float* wp = wpart + (size_t)wid * GT * (D + 2);
+        float* wp = reinterpret_cast<float*>(ring);
 #pragma unroll
         for (int h = 0; h < GT; ++h) {
             if (h >= G) break;
@@ -512,11 +641,14 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     for (int e = tid; e < G * D; e += kNT) {
         const int h = e / D, d = e - h * D;
         float M = -INFINITY;
-        for (int w = 0; w < kNW; ++w) M = fmaxf(M, wpart[(w * GT + h) * (D + 2) + D]);
+        auto wpart = [&](int w) -> const float* {
+            return reinterpret_cast<const float*>(smem + L.region + w * att_ring_bytes(RB)) + h * (D + 2);
+        };
+        for (int w = 0; w < kNW; ++w) M = fmaxf(M, wpart(w)[D]);
         float O = 0.f, Lsum = 0.f;
         if (M != -INFINITY) {
             for (int w = 0; w < kNW; ++w) {
-                const float* wp = wpart + (w * GT + h) * (D + 2);
+                const float* wp = wpart(w);
                 const float f = exp2f(wp[D] - M);
                 O = fmaf(f, wp[d], O);
                 Lsum = fmaf(f, wp[D + 1], Lsum);
@@ -525,6 +657,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         co[h * D + d] = O;
         if (d == 0) { cm[h] = M; cl[h] = Lsum; }
     }
+    // [phase] 8
     cluster.sync();                                            // CTA partials visible
 
     // final merge across the cluster; CTA `rank` writes its slice of [G, D]
@@ -550,6 +683,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
             else reinterpret_cast<float*>(p.out)[oidx] = res;
         }
     }
+    // [phase] 9
     cluster.sync();                                            // keep smem alive for readers
 }
 
