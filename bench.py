@@ -2,14 +2,14 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config I]
 
-One step = one decode token for every sequence of a layer: append the new
-token's heavy channels to the label cache (ds_append_label), then the fused
-decode (ds_sparse_decode: query gather, approximate scores, top-k, exact
-attention over the selected K/V rows). The default workload is the
+One step = one decode token for every sequence of a layer, in one launch
+(ds_decode_step): the new token's heavy channels are appended to the label
+cache, then query gather, approximate scores, top-k and exact attention over
+the selected K/V rows. The default workload is the
 Llama-2-7B-shaped layer (batch 8, 32 MHA heads, head_dim 128, 4096 cached
 tokens, 16 bf16 heavy channels, top-256). Inputs are seeded synthetic tensors.
 
-Timing: CUDA graph per kernel, CUDA events on the launching stream, a 512 MiB
+Timing: the step captured in a CUDA graph, CUDA events on the launching stream, a 512 MiB
 L2-flushing write before every timed step, max over ranks under torchrun
 (weak scaling: every rank runs its own layer; no collective on the data path).
 Rank 0 prints one JSON line.
@@ -58,8 +58,10 @@ def algorithmic_bytes(wl: synth.Workload, out_esz: int = 2) -> dict:
     label = rows * wl.s * lab_row
     kv = rows * k_eff * wl.d * esz * 2
     qo = wl.b * wl.hq * wl.d * (esz + out_esz)
+    append = rows * (wl.d * esz + lab_row)  # new token: key row read, label row written
     dense = rows * wl.s * wl.d * esz * 2 + qo
-    return {"label": label, "kv_selected": kv, "q_out": qo, "total": label + kv + qo, "dense_total": dense}
+    return {"label": label, "kv_selected": kv, "q_out": qo, "append": append,
+            "total": label + kv + qo + append, "dense_total": dense}
 
 
 def measured_peaks() -> dict:
@@ -240,39 +242,32 @@ def run_ours(args, wl, rank, local_rank, world):
     torch.cuda.synchronize()
     prefill_ms = e0.elapsed_time(e1)
 
-    def append():
-        ds.append_label(k, idx, pos, lab, sc, ze)
-
-    def decode():
-        ds.sparse_decode(q, k, v, lab, idx, wl.s, wl.topk, lscale=sc, lzero=ze, out=out)
+    def step():
+        # one launch: label row of token s-1 (ds_append_label's work) + sparse decode
+        ds.decode_step(q, k, v, lab, idx, wl.s, wl.topk, lscale=sc, lzero=ze, out=out)
 
     with torch.cuda.stream(stream):
         for _ in range(3):  # set kernel attributes before capture
-            append(); decode()
+            step()
     stream.synchronize()
-    g_app, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_app, stream=stream):
-        append()
-    with torch.cuda.graph(g_dec, stream=stream):
-        decode()
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step, stream=stream):
+        step()
 
     def one_step(evs=None):
-        flush.zero_()  # untimed: evicts L2 (inputs of c1 fit in the 126 MB L2)
+        flush.zero_()  # untimed: evicts L2 (the step's inputs could otherwise stay in the 126 MB L2)
         if evs:
             evs[0].record()
-        g_app.replay()
+        g_step.replay()
         if evs:
             evs[1].record()
-        g_dec.replay()
-        if evs:
-            evs[2].record()
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             one_step()
     torch.cuda.synchronize()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     sampler = ClockSampler(local_rank)
     barrier()
     torch.cuda.synchronize()
@@ -284,9 +279,7 @@ def run_ours(args, wl, rank, local_rank, world):
         torch.cuda.synchronize()
         wall1 = time.perf_counter()
     barrier()
-    step_ms = [e[0].elapsed_time(e[2]) for e in evs]
-    dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    app_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    step_ms = [e[0].elapsed_time(e[1]) for e in evs]
     total_s = sum(step_ms) / 1e3
     max_s = reduce_max(total_s, dev)
 
@@ -310,8 +303,7 @@ def run_ours(args, wl, rank, local_rank, world):
             dv.copy_(hv, non_blocking=True)
             k[:, :, pos].copy_(dk)
             v[:, :, pos].copy_(dv)
-            ds.append_label(k, idx, pos, lab, sc, ze)
-            ds.sparse_decode(dq, k, v, lab, idx, wl.s, wl.topk, lscale=sc, lzero=ze, out=out)
+            ds.decode_step(dq, k, v, lab, idx, wl.s, wl.topk, lscale=sc, lzero=ze, out=out)
             hout.copy_(out, non_blocking=True)
             b_.record()
             if i >= args.warmup:
@@ -325,7 +317,7 @@ def run_ours(args, wl, rank, local_rank, world):
     # dense baseline on the same cache: our dense kernel and torch SDPA
     dense_ms, sdpa_ms = dense_baselines(wl, q, k, v, out, flush, stream)
 
-    res = dict(step_ms=step_ms, dec_ms=dec_ms, app_ms=app_ms, total_s=total_s, max_s=max_s,
+    res = dict(step_ms=step_ms, total_s=total_s, max_s=max_s,
                wall_s=wall1 - wall0, e2e_s=e2e_max, h2d=h2d, d2h=d2h, prefill_ms=prefill_ms,
                clocks=sampler.summary(), dense_ms=dense_ms, sdpa_ms=sdpa_ms,
                plan=ds.plan(wl.b, wl.hq, wl.hkv, wl.s, wl.d, wl.c, wl.topk,
@@ -501,9 +493,8 @@ def report(args, wl, r, world):
     ab = algorithmic_bytes(wl, r["out_esz"])
     peaks = measured_peaks()
     value = job_value(wl.b, world, args.steps, r["max_s"])
-    dec_avg_s = sum(r["dec_ms"]) / len(r["dec_ms"]) / 1e3
+    dec_avg_s = sum(r["step_ms"]) / len(r["step_ms"]) / 1e3  # the step is one launch of the kernel
     achieved = ab["total"] / dec_avg_s / 1e9
-    step_avg_s = sum(r["step_ms"]) / len(r["step_ms"]) / 1e3
     cpu = None
     if world == 1:
         host = host_arrays(wl, r["host"])
@@ -524,12 +515,11 @@ def report(args, wl, r, world):
                      "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"],
                      "traffic": recorded_traffic(args.config), "kernel": "ds_decode_kernel",
                      "algorithmic_bytes_per_launch": ab["total"], "avg_launch_us": dec_avg_s * 1e6},
-        "step_breakdown_us": {"append_label": 1e6 * sum(r["app_ms"]) / len(r["app_ms"]) / 1e3,
-                              "sparse_decode": dec_avg_s * 1e6, "step": step_avg_s * 1e6},
+        "step_us": dec_avg_s * 1e6,
         "cpu_baseline": cpu,
         "e2e": {"value": job_value(wl.b, world, args.steps, r["e2e_s"]), "unit": UNIT,
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": args.steps,
         "clocks": r["clocks"],
         "dense_baseline": {"ds_dense_decode_us": r["dense_ms"] * 1e3,
                            "torch_sdpa_us": None if r["sdpa_ms"] is None else r["sdpa_ms"] * 1e3,

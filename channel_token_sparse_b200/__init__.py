@@ -35,6 +35,8 @@ SIGNATURES = {
     "ds_append_label": (_i, [_vp, _i, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _vp]),
     "ds_sparse_decode": (_i, [_vp, _vp, _vp, _i, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
                               _f, _vp, _i, _vp, _vp, _vp]),
+    "ds_decode_step": (_i, [_vp, _vp, _vp, _i, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
+                            _f, _vp, _i, _vp, _vp, _vp]),
     "ds_sparse_decode_plan": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, _i, C.POINTER(_i), C.POINTER(_i),
                                    C.POINTER(_i)]),
     "ds_sparse_decode_set_cluster": (None, [_i]),
@@ -216,6 +218,26 @@ def sparse_decode(q, k, v, label, idx, s: int, topk: int, lscale=None, lzero=Non
                                   _label_args(label, lscale, lzero, kdt), _ptr(lscale), _ptr(lzero),
                                   _ptr(idx), b, hq, hkv, s, s_cap, d, c, topk, float(sm_scale),
                                   _ptr(out), odt, _ptr(sel_out), _ptr(score_out), _stream(stream)))
+    return out
+
+
+def decode_step(q, k, v, label, idx, s: int, topk: int, lscale=None, lzero=None, out=None,
+                out_dtype=None, sm_scale: float = 0.0, sel_out=None, score_out=None, stream=None):
+    """append_label(pos = s - 1) followed by sparse_decode, in one launch;
+    returns out [B, Hq, D]."""
+    torch = _torch()
+    _need_cuda(q, k, v, label, idx, lscale, lzero, out, sel_out, score_out)
+    b, hq, d = q.shape
+    _, hkv, s_cap, _ = k.shape
+    c = idx.shape[1]
+    kdt = _kv_dtype(k)
+    if out is None:
+        out = torch.empty((b, hq, d), dtype=out_dtype or torch.float32, device=q.device)
+    odt = DS_F32 if out.dtype == torch.float32 else DS_BF16
+    _check(lib().ds_decode_step(_ptr(q), _ptr(k), _ptr(v), kdt, _ptr(label),
+                                _label_args(label, lscale, lzero, kdt), _ptr(lscale), _ptr(lzero),
+                                _ptr(idx), b, hq, hkv, s, s_cap, d, c, topk, float(sm_scale),
+                                _ptr(out), odt, _ptr(sel_out), _ptr(score_out), _stream(stream)))
     return out
 
 

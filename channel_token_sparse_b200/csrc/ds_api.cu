@@ -47,6 +47,17 @@ int sm_count() {
     return n;
 }
 
+// L2 size of the current device (126 MB on B200); queried once per process.
+int l2_bytes() {
+    static int n = [] {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return 126 << 20;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrL2CacheSize, dev) != cudaSuccess) return 126 << 20;
+        return v > 0 ? v : 126 << 20;
+    }();
+    return n;
+}
+
 constexpr int kMaxSmem = 227 * 1024;
 constexpr int kCtasPerSm = 2;  // __launch_bounds__(256, 2) -> <= 128 registers
 
@@ -252,11 +263,15 @@ ds_status ds_sparse_decode_plan(int b, int hq, int hkv, int s, int d, int c, int
     return DS_OK;
 }
 
-ds_status ds_sparse_decode(const void* q, const void* k, const void* v, ds_dtype kvdt,
-                           const void* label, ds_dtype label_dt, const uint16_t* lscale,
-                           const uint16_t* lzero, const int32_t* idx, int b, int hq, int hkv, int s,
-                           int s_cap, int d, int c, int topk, float sm_scale, void* out,
-                           ds_dtype out_dt, int32_t* sel_out, float* score_out, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+ds_status sparse_decode_impl(const void* q, const void* k, const void* v, ds_dtype kvdt, const void* label,
+                             ds_dtype label_dt, const uint16_t* lscale, const uint16_t* lzero,
+                             const int32_t* idx, int b, int hq, int hkv, int s, int s_cap, int d, int c,
+                             int topk, float sm_scale, void* out, ds_dtype out_dt, int32_t* sel_out,
+                             float* score_out, bool append, cudaStream_t stream) {
     ds_status r = check_common(b, hq, hkv, s, s_cap, d, kvdt);
     if (r != DS_OK) return r;
     if ((r = check_label(kvdt, label_dt, c, d, label, lscale, lzero)) != DS_OK) return r;
@@ -281,11 +296,34 @@ ds_status ds_sparse_decode(const void* q, const void* k, const void* v, ds_dtype
     p.out = out; p.sel_out = sel_out; p.score_out = score_out;
     p.hkv = hkv; p.G = G; p.s = s; p.s_cap = s_cap; p.topk = topk;
     p.chunk = pl.chunk; p.lay_chunk = pl.lay_chunk; p.per = pl.per;
+    p.append = append ? 1 : 0;
     const float scale = sm_scale > 0.f ? sm_scale : 1.0f / sqrtf((float)d);
     p.qscale = scale * 1.4426950408889634f;
     p.out_bf16 = out_dt == DS_BF16;
     p.dense = 0;
     return launch_decode(kern, p, rows, pl, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+ds_status ds_sparse_decode(const void* q, const void* k, const void* v, ds_dtype kvdt,
+                           const void* label, ds_dtype label_dt, const uint16_t* lscale,
+                           const uint16_t* lzero, const int32_t* idx, int b, int hq, int hkv, int s,
+                           int s_cap, int d, int c, int topk, float sm_scale, void* out,
+                           ds_dtype out_dt, int32_t* sel_out, float* score_out, cudaStream_t stream) {
+    return sparse_decode_impl(q, k, v, kvdt, label, label_dt, lscale, lzero, idx, b, hq, hkv, s, s_cap, d, c,
+                              topk, sm_scale, out, out_dt, sel_out, score_out, false, stream);
+}
+
+ds_status ds_decode_step(const void* q, const void* k, const void* v, ds_dtype kvdt, void* label,
+                         ds_dtype label_dt, uint16_t* lscale, uint16_t* lzero, const int32_t* idx, int b,
+                         int hq, int hkv, int s, int s_cap, int d, int c, int topk, float sm_scale,
+                         void* out, ds_dtype out_dt, int32_t* sel_out, float* score_out,
+                         cudaStream_t stream) {
+    return sparse_decode_impl(q, k, v, kvdt, label, label_dt, lscale, lzero, idx, b, hq, hkv, s, s_cap, d, c,
+                              topk, sm_scale, out, out_dt, sel_out, score_out, true, stream);
 }
 
 ds_status ds_dense_decode(const void* q, const void* k, const void* v, ds_dtype kvdt, int b, int hq,

@@ -96,6 +96,111 @@ __device__ __forceinline__ void lds_words(uint32_t (&w)[N / 4], const uint8_t* p
     }
 }
 
+// Shared-memory loads of a label row of N bytes (N a multiple of 4).
+template <int N>
+__device__ __forceinline__ void lds_row(uint32_t (&w)[N / 4], const uint8_t* p) {
+    if constexpr (N % 16 == 0) {
+#pragma unroll
+        for (int i = 0; i < N / 16; ++i) {
+            const uint4 x = reinterpret_cast<const uint4*>(p)[i];
+            w[4 * i + 0] = x.x; w[4 * i + 1] = x.y; w[4 * i + 2] = x.z; w[4 * i + 3] = x.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < N / 4; ++i) w[i] = reinterpret_cast<const uint32_t*>(p)[i];
+    }
+}
+
+// 4-bit label row of one token (the heavy channels idx[0..c) of key row x):
+// in fp32, mn/mx over the c values, scale = fp16_rn((mx - mn) / 15),
+// zero = fp16_rn(mn), code_j = scale > 0 ? clamp(rint((x_j - zero) / scale),
+// 0, 15) : 0 with IEEE division and round-half-even; channel 2j goes to the
+// low nibble of byte j. Used by the label kernel and by the fused decode step,
+// so both produce the same bits.
+template <typename T>
+__device__ __forceinline__ void pack_int4_row(const T* x, const int* idx, int c, uint8_t* payload,
+                                              uint16_t* scale_bits, uint16_t* zero_bits) {
+    float mn = Elem<T>::to_f32(x[idx[0]]), mx = mn;
+    for (int j = 1; j < c; ++j) {
+        const float v = Elem<T>::to_f32(x[idx[j]]);
+        mn = fminf(mn, v);
+        mx = fmaxf(mx, v);
+    }
+    const float step = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+    const uint16_t sh = __half_as_ushort(__float2half_rn(step));
+    const uint16_t zh = __half_as_ushort(__float2half_rn(mn));
+    const float sc = fp16_bits_to_f32(sh);
+    const float z = fp16_bits_to_f32(zh);
+    for (int j = 0; j < c; j += 2) {
+        uint32_t nib[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            uint32_t code = 0;
+            if (sc > 0.f) {
+                float qv = rintf(__fdiv_rn(__fsub_rn(Elem<T>::to_f32(x[idx[j + e]]), z), sc));
+                qv = fminf(fmaxf(qv, 0.f), 15.f);
+                code = (uint32_t)qv;
+            }
+            nib[e] = code;
+        }
+        payload[j / 2] = (uint8_t)(nib[0] | (nib[1] << 4));
+    }
+    *scale_bits = sh;
+    *zero_bits = zh;
+}
+
+// Sum NV values (NV a power of two, <= 32) over the 32 lanes of a warp; on
+// return every lane holds all NV sums. A transposing butterfly: at each of
+// the first log2(NV) exchange steps a lane sends half of its values and keeps
+// the other half, so NV - 1 + 5 - log2(NV) shuffles reduce, and NV shuffles
+// broadcast (instead of 5 * NV for separate reductions).
+template <int NV>
+__device__ __forceinline__ void warp_allreduce_multi(float (&v)[NV]) {
+    constexpr int LOGN = NV >= 32 ? 5 : NV >= 16 ? 4 : NV >= 8 ? 3 : NV >= 4 ? 2 : NV >= 2 ? 1 : 0;
+    static_assert((1 << LOGN) == NV, "NV must be a power of two <= 32");
+    const int lane = threadIdx.x & 31;
+    float r[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) r[i] = v[i];
+#pragma unroll
+    for (int step = 0; step < 5; ++step) {
+        const int m = 16 >> step;
+        if (step < LOGN) {
+            const int half = NV >> (step + 1);
+            const bool up = (lane & m) != 0;
+#pragma unroll
+            for (int i = 0; i < half; ++i) {
+                const float send = up ? r[i] : r[i + half];
+                const float keep = up ? r[i + half] : r[i];
+                r[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+            }
+        } else {
+            r[0] += __shfl_xor_sync(0xffffffffu, r[0], m);
+        }
+    }
+    // lane l now holds the sum of value (l >> (5 - LOGN))
+#pragma unroll
+    for (int j = 0; j < NV; ++j) v[j] = __shfl_sync(0xffffffffu, r[0], j << (5 - LOGN));
+}
+
+// Same for any power of two NV: blocks of 32 values at a time.
+template <int NV>
+__device__ __forceinline__ void warp_allreduce_n(float (&v)[NV]) {
+    if constexpr (NV <= 32) {
+        warp_allreduce_multi<NV>(v);
+    } else {
+#pragma unroll
+        for (int b = 0; b < NV / 32; ++b) {
+            float t[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) t[i] = v[b * 32 + i];
+            warp_allreduce_multi<32>(t);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[b * 32 + i] = t[i];
+        }
+    }
+}
+
 // 16-byte asynchronous global -> shared copy (LDGSTS, L2 only), and its
 // group bookkeeping. Completion is awaited per thread with cp_async_wait;
 // other lanes' copies become visible after a __syncwarp / __syncthreads.
@@ -107,25 +212,9 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// Bulk prefetch of [p, p + bytes) into L2 (TMA unit; no registers held while
-// in flight). p must be 16-byte aligned and bytes a multiple of 16.
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
-// Prefetch the byte range [base + lo, base + hi) in pieces of `piece` bytes
-// (a multiple of 16), one piece per thread index `who`. The range is trimmed
-// inward to 16-byte aligned ABSOLUTE addresses (row bases of small-row arrays,
-// e.g. fp16 scales at row * s_cap * 2 bytes, need not be aligned), so every
-// prefetch starts on a 16-byte boundary and covers a multiple of 16 bytes.
-__device__ __forceinline__ void prefetch_range(const uint8_t* base, size_t lo, size_t hi, int who,
-                                               uint32_t piece) {
-    const uintptr_t a = (reinterpret_cast<uintptr_t>(base + lo) + 15) & ~(uintptr_t)15;
-    const uintptr_t e = reinterpret_cast<uintptr_t>(base + hi) & ~(uintptr_t)15;
-    const uintptr_t start = a + (uintptr_t)who * piece;
-    if (start >= e) return;
-    const uintptr_t n = e - start < piece ? e - start : piece;
-    prefetch_l2(reinterpret_cast<const void*>(start), (uint32_t)n);
+// Prefetch of the 128-byte line holding p into L2 (no register result).
+__device__ __forceinline__ void prefetch_line_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 // Order-preserving map of an fp32 score to uint32: larger score -> larger key.

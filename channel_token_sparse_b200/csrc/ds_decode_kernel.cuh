@@ -37,8 +37,6 @@ constexpr int kNW = kNT / 32;        // warps per CTA
 constexpr int kMaxChunk = 32768;     // tokens per CTA (16-bit keys -> 64 KiB)
 constexpr int kLabelInt4 = 1;
 constexpr int kLabelFp = 0;
-constexpr uint32_t kPfPiece = 4096;  // bytes per L2 bulk-prefetch instruction
-constexpr int kPfRounds = 2;         // scoring rounds prefetched ahead
 
 struct DecodeParams {
     const void* q;
@@ -55,6 +53,7 @@ struct DecodeParams {
     int chunk;     // tokens per CTA, multiple of 32
     int lay_chunk; // chunk used to size shared memory (0 in dense mode)
     int per;       // selected tokens attended per CTA (ceil(min(topk,s) / N))
+    int append;    // 1: first build the label row of token s-1 from the key cache (decode step)
     float qscale;  // sm_scale * log2(e)
     int out_bf16;
     int dense;     // 1: attend every token, no label / scores / selection
@@ -62,7 +61,7 @@ struct DecodeParams {
 
 // Shared-memory carve-up (bytes), identical on host and device.
 struct DecodeSmem {
-    int qs, qL, idx, histA, histB, ctl, scan, cm, cl, co, bits, blist, sel, region, total;
+    int qs, qL, idx, histA, histB, ctl, scan, cm, cl, co, bits, blist, app, sel, region, total;
 };
 
 __host__ __device__ inline int align16(int x) { return (x + 15) & ~15; }
@@ -98,6 +97,7 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int GT, int D, int C, i
     L.co = o;     o += align16(GT * D * 4);
     L.bits = o;   o += align16(chunk / 8);
     L.blist = o;  o += chunk > 0 ? kBucketCap * 4 : 0;
+    L.app = o;    o += align16(C * 4) + 16;  // appended token's label row (+ fp16 scale, zero)
     L.sel = o;    o += align16(per * 4);
     L.region = o;
     const int keys = chunk * 2;
@@ -156,6 +156,18 @@ __device__ __forceinline__ float label_score(const uint32_t (&w)[LabelGeom<TKV, 
     }
 }
 
+// Barrier and shared-memory mapping across the CTAs of a row: a single-CTA
+// cluster (N == 1, uniform per launch) uses the CTA barrier and plain
+// shared-memory pointers instead of the cluster barrier and DSMEM windows.
+__device__ __forceinline__ void row_sync(cg::cluster_group& cluster, int nblocks) {
+    if (nblocks == 1) __syncthreads();
+    else cluster.sync();
+}
+template <typename T>
+__device__ __forceinline__ T* row_smem(cg::cluster_group& cluster, int nblocks, T* p, int rank) {
+    return nblocks == 1 ? p : cluster.map_shared_rank(p, rank);
+}
+
 // Sum a 256-bin histogram over the cluster (DSMEM) and find the bin holding
 // the `need`-th largest key. Writes ctl[kCtlBin], ctl[kCtlNeed] (how many to
 // take from that bin) and ctl[kCtlCnt] (the bin's size). Requires a cluster
@@ -169,7 +181,7 @@ __device__ __forceinline__ void cluster_select_bin(cg::cluster_group& cluster, u
     const int tid = threadIdx.x;
     const int bin = 255 - tid;  // thread 0 holds the largest bin
     uint32_t cnt = 0;
-    for (int r = 0; r < nblocks; ++r) cnt += cluster.map_shared_rank(hist, r)[bin];
+    for (int r = 0; r < nblocks; ++r) cnt += row_smem(cluster, nblocks, hist, r)[bin];
     if (zero_next) zero_next[tid] = 0u;
     uint32_t total;
     const uint32_t excl = block_excl_scan<kNT>(cnt, scan, &total);
@@ -229,18 +241,6 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     const bool need_scores = !p.dense && (!select_all || p.score_out != nullptr);
     constexpr int U = LG::kU;
     constexpr int kRound = kNT * U;  // tokens per scoring round
-    // Start pulling the first rounds of this CTA's label rows into L2 while
-    // the query is set up; the scoring loop keeps kPfRounds rounds ahead.
-    auto prefetch_label_round = [&](int r) {
-        const size_t lo = (size_t)(t0 + r * kRound), hi = (size_t)(t0 + min(n_loc, (r + 1) * kRound));
-        if (r * kRound >= n_loc) return;
-        constexpr int kPieces = (kRound * LG::kBytes + kPfPiece - 1) / kPfPiece;
-        if (tid < kPieces) prefetch_range(lab, lo * LG::kBytes, hi * LG::kBytes, tid, kPfPiece);
-        if constexpr (LK == kLabelInt4) {
-            if (tid == kPieces) prefetch_range(reinterpret_cast<const uint8_t*>(lsc), lo * 2, hi * 2, 0, kRound * 2);
-            if (tid == kPieces + 1) prefetch_range(reinterpret_cast<const uint8_t*>(lze), lo * 2, hi * 2, 0, kRound * 2);
-        }
-    };
 
     // ---------------------------------------------------------- setup, step 1
     for (int e = tid; e < G * D; e += kNT) qs[e] = E::to_f32(qrow[e]);
@@ -250,8 +250,6 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         histB[tid] = 0u;
         if (tid == 0) ctl[kCtlBL] = 0;
     }
-    if (need_scores)  // after the q / idx loads, so they do not queue behind it
-        for (int r = 0; r <= kPfRounds; ++r) prefetch_label_round(r);
     __syncthreads();
     if (!p.dense) {
         for (int j = tid; j < C; j += kNT) {
@@ -260,21 +258,56 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
             qLs[j] = a;
         }
     }
+    // decode step: the CTA holding token s-1 builds its label row (the same
+    // copy / 4-bit pack as ds_append_label), keeps it in shared memory and
+    // stores it to the label cache
+    const int app_i = (p.append && !p.dense && s - 1 >= t0 && s - 1 < t0 + n_loc) ? s - 1 - t0 : -1;
+    if (app_i >= 0 && wid == 0) {
+        const TKV* krow = reinterpret_cast<const TKV*>(p.k) + (row_tok + (size_t)(s - 1)) * D;
+        uint8_t* grow = const_cast<uint8_t*>(lab) + (size_t)(s - 1) * LG::kBytes;
+        if constexpr (LK == kLabelFp) {
+            TKV* srow = reinterpret_cast<TKV*>(smem + L.app);
+            for (int j = lane; j < C; j += 32) {
+                const TKV x = krow[idx_s[j]];
+                srow[j] = x;
+                reinterpret_cast<TKV*>(grow)[j] = x;
+            }
+        } else if (lane == 0) {
+            uint16_t* ssz = reinterpret_cast<uint16_t*>(smem + L.app + align16(C * 4));
+            pack_int4_row<TKV>(krow, idx_s, C, smem + L.app, &ssz[0], &ssz[1]);
+            for (int j = 0; j < C / 2; ++j) grow[j] = smem[L.app + j];
+            const_cast<uint16_t*>(lsc)[s - 1] = ssz[0];
+            const_cast<uint16_t*>(lze)[s - 1] = ssz[1];
+        }
+    }
     __syncthreads();
 
     float qreg[C <= 32 ? C : 1];
     float qsum = 0.f;
 
-    // Score of token t (absolute index in the row) straight from global memory;
-    // same arithmetic as the streaming loop below.
-    auto rescore = [&](int t) -> float {
-        uint32_t w[LG::kWords];
-        load_words<LG::kBytes>(w, lab + (size_t)t * LG::kBytes);
-        float sc = 0.f, z = 0.f;
-        if constexpr (LK == kLabelInt4) {
-            sc = fp16_bits_to_f32(ldg_u16(lsc + t));
-            z = fp16_bits_to_f32(ldg_u16(lze + t));
+    // The label row of the appended token (local index app_i, -1 if none) is
+    // read from shared memory: this kernel writes it to the label cache and
+    // must not read it back through the read-only path.
+    const uint8_t* app_row = smem + L.app;
+    const uint16_t* app_sz = reinterpret_cast<const uint16_t*>(smem + L.app + align16(C * 4));
+    auto load_label = [&](int i, uint32_t (&w)[LG::kWords], float& sc, float& z) {
+        if (i == app_i) {
+            lds_row<LG::kBytes>(w, app_row);
+            if constexpr (LK == kLabelInt4) { sc = fp16_bits_to_f32(app_sz[0]); z = fp16_bits_to_f32(app_sz[1]); }
+        } else {
+            load_words<LG::kBytes>(w, lab + (size_t)(t0 + i) * LG::kBytes);
+            if constexpr (LK == kLabelInt4) {
+                sc = fp16_bits_to_f32(ldg_u16(lsc + t0 + i));
+                z = fp16_bits_to_f32(ldg_u16(lze + t0 + i));
+            }
         }
+    };
+    // Score of local token i straight from memory; same arithmetic as the
+    // streaming loop below.
+    auto rescore = [&](int i) -> float {
+        uint32_t w[LG::kWords];
+        float sc = 0.f, z = 0.f;
+        load_label(i, w, sc, z);
         return label_score<TKV, LK, C>(w, qreg, qLs, sc, z, qsum);
     };
 
@@ -290,19 +323,12 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     // ---------------------------------------------------------------- step 2
     if (need_scores) {
         for (int base = 0; base < n_loc; base += kRound) {
-            prefetch_label_round(base / kRound + kPfRounds + 1);
             uint32_t w[U][LG::kWords];
             float sc[U], z[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int i = base + u * kNT + tid;
-                if (i < n_loc) {
-                    load_words<LG::kBytes>(w[u], lab + (size_t)(t0 + i) * LG::kBytes);
-                    if constexpr (LK == kLabelInt4) {
-                        sc[u] = fp16_bits_to_f32(ldg_u16(lsc + t0 + i));
-                        z[u] = fp16_bits_to_f32(ldg_u16(lze + t0 + i));
-                    }
-                }
+                if (i < n_loc) load_label(i, w[u], sc[u], z[u]);
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
@@ -327,10 +353,13 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
 
     // [phase] 2
     // --------------------------------------------------------------- step 3a
+    const TKV* kb = reinterpret_cast<const TKV*>(p.k) + row_tok * D;
+    const TKV* vb = reinterpret_cast<const TKV*>(p.v) + row_tok * D;
+    constexpr int RB = D * E::kBytes;              // bytes of one K or V row
     int T16 = 0, Tlo = 0, r_tie = 0;
     bool refine = false;
     if (!select_all) {
-        cluster.sync();                                        // histograms A complete
+        row_sync(cluster, N);                                        // histograms A complete
         cluster_select_bin(cluster, histA, N, (uint32_t)k_eff, ctl, scan, nullptr);
         const int bA = ctl[kCtlBin];
         const int needA = ctl[kCtlNeed];
@@ -351,7 +380,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
             }
         }
         // [phase] 10
-        cluster.sync();                                        // histograms B complete
+        row_sync(cluster, N);                                        // histograms B complete
         // [phase] 11
         cluster_select_bin(cluster, histB, N, (uint32_t)needA, ctl, scan, histA);
         T16 = (bA << 8) | ctl[kCtlBin];
@@ -372,7 +401,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
                 bits8[grp] = (uint8_t)flags;
                 for (uint32_t m = flags; m; m &= m - 1) {
                     const int i = grp * 8 + __ffs(m) - 1;
-                    const uint32_t low = score_key(rescore(t0 + i)) & 0xFFFFu;
+                    const uint32_t low = score_key(rescore(i)) & 0xFFFFu;
                     keys[i] = (uint16_t)low;
                     atomicAdd(&histA[low >> 8], 1u);
                     const int slot = atomicAdd(&ctl[kCtlBL], 1);
@@ -380,7 +409,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
                 }
             }
             // [phase] 12
-            cluster.sync();                                    // histograms C complete
+            row_sync(cluster, N);                                    // histograms C complete
             // [phase] 13
             cluster_select_bin(cluster, histA, N, (uint32_t)needB, ctl, scan, histB);
             const int bC = ctl[kCtlBin];
@@ -405,7 +434,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
                 }
             }
             // [phase] 14
-            cluster.sync();                                    // histograms D complete
+            row_sync(cluster, N);                                    // histograms D complete
             // [phase] 15
             cluster_select_bin(cluster, histB, N, (uint32_t)needC, ctl, scan, nullptr);
             Tlo = (bC << 8) | ctl[kCtlBin];
@@ -418,33 +447,32 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         // Warp w owns a contiguous segment of key groups; in each step lane l
         // reads group seg + 32*step + l (conflict-free 16-byte loads), so lane
         // order is index order and warp scans rank the selected tokens.
-        auto klass = [&](int k16, bool inb) -> int {
-            if (!refine) return k16 >= T16 ? 1 : 0;
-            if (inb) return k16 > Tlo ? 1 : (k16 == Tlo ? 2 : 0);
-            return k16 > T16 ? 1 : 0;
-        };
-        // per group: strict count in bits 0..7, tie count in bits 8..15, and
-        // the class of each of its 8 keys (2 bits each) in bits 16..31
-        auto classify8 = [&](int grp) -> uint32_t {
-            if (grp >= ngrp) return 0u;
+        // Per key group: bit e of the low byte marks a key selected outright,
+        // bit e of the second byte an exact tie with the k-th key.
+        auto masks8 = [&](int grp) -> uint32_t {
             uint32_t w[4];
             key8(grp, w);
             const uint32_t fl = refine ? bits8[grp] : 0u;
-            uint32_t r = 0;
+            const int lim = n_loc - grp * 8;
+            uint32_t sm = 0, tm = 0;
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const uint32_t c = grp * 8 + e < n_loc ? (uint32_t)klass(kat(w, e), (fl >> e) & 1u) : 0u;
-                r += (c == 1u) + ((c == 2u) << 8) + (c << (16 + 2 * e));
+                const int k16 = kat(w, e);
+                const bool inb = (fl >> e) & 1u;
+                const bool strict = refine ? k16 > (inb ? Tlo : T16) : k16 >= T16;
+                const bool tie = inb && k16 == Tlo;
+                sm |= (uint32_t)(e < lim && strict) << e;
+                tm |= (uint32_t)(e < lim && tie) << e;
             }
-            return r;
+            return sm | (tm << 8);
         };
         const int gpw = (((ngrp + kNW - 1) / kNW) + 31) & ~31;   // groups per warp
         const int wg0 = wid * gpw, wg1 = min(ngrp, wg0 + gpw);
         uint32_t ns = 0, nt = 0;
         for (int grp = wg0 + lane; grp - lane < wg1; grp += 32) {
-            const uint32_t r = grp < wg1 ? classify8(grp) : 0u;
-            ns += r & 255u;
-            nt += (r >> 8) & 255u;
+            const uint32_t m = grp < wg1 ? masks8(grp) : 0u;
+            ns += __popc(m & 255u);
+            nt += __popc(m >> 8);
         }
         ns = (uint32_t)__reduce_add_sync(0xffffffffu, ns);
         nt = (uint32_t)__reduce_add_sync(0xffffffffu, nt);
@@ -459,12 +487,12 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         }
         // [phase] 16
         // [phase] 17
-        cluster.sync();                                        // per-CTA counts visible
+        row_sync(cluster, N);                                        // per-CTA counts visible
         // [phase] 18
         if (wid == 0) {
             int cs = 0, ct = 0;
             if (lane < N) {
-                const int* rc = cluster.map_shared_rank(ctl, lane);
+                const int* rc = row_smem(cluster, N, ctl, lane);
                 cs = rc[kCtlCS];
                 ct = rc[kCtlCT];
             }
@@ -480,32 +508,36 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         const int P = ctl[kCtlP], TP = ctl[kCtlTP];
         const int tie_quota = max(0, r_tie - TP);  // ties this CTA may still take
         int sb = (int)(scan[wid] >> 16), tb = (int)(scan[wid] & 0xFFFFu);  // before this step
-        const int per = p.per;
+        const uint32_t per = (uint32_t)p.per;
+        const uint32_t per_inv = 0xFFFFFFFFu / per;  // q = umulhi(pos, per_inv) is q or q-1
+        int cur_dst = -1;
+        int* rl = nullptr;
         for (int grp = wg0 + lane; grp - lane < wg1; grp += 32) {
-            const uint32_t r = grp < wg1 ? classify8(grp) : 0u;
-            const uint32_t cs_l = r & 255u, ct_l = (r >> 8) & 255u;
-            const uint32_t pk = (cs_l << 16) | ct_l;
+            const uint32_t m = grp < wg1 ? masks8(grp) : 0u;
+            const uint32_t smk = m & 255u, tmk = m >> 8;
+            const uint32_t pk = ((uint32_t)__popc(smk) << 16) | (uint32_t)__popc(tmk);
             const uint32_t incl = warp_incl_scan(pk);
-            int my_sb = sb + (int)((incl - pk) >> 16), my_tb = tb + (int)((incl - pk) & 0xFFFFu);
+            const int my_sb = sb + (int)((incl - pk) >> 16), my_tb = tb + (int)((incl - pk) & 0xFFFFu);
             const uint32_t tot_step = __shfl_sync(0xffffffffu, incl, 31);
             sb += (int)(tot_step >> 16);
             tb += (int)(tot_step & 0xFFFFu);
-            for (uint32_t cls = r >> 16, e = 0; cls; cls >>= 2, ++e) {
-                const uint32_t c = cls & 3u;
-                if (c == 1u || (c == 2u && my_tb < tie_quota)) {
-                    const int pos = P + my_sb + min(my_tb, tie_quota);
-                    const int dst = pos / per;
-                    int* rl = cluster.map_shared_rank(sel_list, dst);
-                    const int t = t0 + grp * 8 + (int)e;
-                    rl[pos - dst * per] = t;
-                    if (p.sel_out) p.sel_out[(size_t)row * p.topk + pos] = t;
-                }
-                my_sb += c == 1u;
-                my_tb += c == 2u;
+            for (uint32_t mm = smk | tmk; mm; mm &= mm - 1u) {
+                const int e = __ffs(mm) - 1;
+                const uint32_t below = (1u << e) - 1u;
+                const int s_before = my_sb + __popc(smk & below);
+                const int t_before = my_tb + __popc(tmk & below);
+                if (((tmk >> e) & 1u) && t_before >= tie_quota) continue;  // tie beyond the quota
+                const uint32_t pos = (uint32_t)(P + s_before + min(t_before, tie_quota));
+                uint32_t dst = __umulhi(pos, per_inv);
+                if ((dst + 1u) * per <= pos) ++dst;
+                if ((int)dst != cur_dst) { cur_dst = (int)dst; rl = row_smem(cluster, N, sel_list, (int)dst); }
+                const int t = t0 + grp * 8 + e;
+                rl[pos - dst * per] = t;
+                if (p.sel_out) p.sel_out[(size_t)row * p.topk + pos] = t;
             }
         }
         // [phase] 20
-        cluster.sync();                                        // selection lists complete
+        row_sync(cluster, N);                                        // selection lists complete
     } else if (p.sel_out) {
         for (int i = tid; i < n_loc; i += kNT) p.sel_out[(size_t)row * p.topk + t0 + i] = t0 + i;
         if (rank == 0)
@@ -517,9 +549,6 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     // Each warp streams the K and V rows of its tokens through a ring of
     // kAttStages shared-memory stages with cp.async (16-byte LDGSTS, no
     // registers held while in flight), kAttStages-1 stages ahead of compute.
-    const TKV* kb = reinterpret_cast<const TKV*>(p.k) + row_tok * D;
-    const TKV* vb = reinterpret_cast<const TKV*>(p.v) + row_tok * D;
-    constexpr int RB = D * E::kBytes;              // bytes of one K or V row
     constexpr int TBS = att_stage_tokens(RB);      // tokens per stage
     constexpr int kStageBytes = 2 * TBS * RB;
     constexpr int kPiecesPerRow = RB / 16;
@@ -571,7 +600,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         const uint8_t* st = ring + (bi % kAttStages) * kStageBytes;
         const int bt0 = (wid + bi * kNW) * TBS;
         bool ok[TBS];
-        float zt[TBS][GT];
+        float zt[TBS * GT];  // index u * GT + h
 #pragma unroll
         for (int u = 0; u < TBS; ++u) {
             ok[u] = bt0 + u < n_att;
@@ -588,15 +617,16 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
                 float a = 0.f;
 #pragma unroll
                 for (int e = 0; e < EPL; ++e) a = fmaf(qf[h][e], kf[e], a);
-                zt[u][h] = warp_sum(a);
+                zt[u * GT + h] = a;
             }
         }
+        warp_allreduce_n<TBS * GT>(zt);
 #pragma unroll
         for (int h = 0; h < GT; ++h) {
             if (h >= G) break;
             float mx = -INFINITY;
 #pragma unroll
-            for (int u = 0; u < TBS; ++u) if (ok[u]) mx = fmaxf(mx, zt[u][h]);
+            for (int u = 0; u < TBS; ++u) if (ok[u]) mx = fmaxf(mx, zt[u * GT + h]);
             const float m_new = fmaxf(m_run[h], mx);
             const float corr = exp2f(m_run[h] - m_new);
             float l = l_run[h] * corr;
@@ -605,7 +635,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
 #pragma unroll
             for (int u = 0; u < TBS; ++u) {
                 if (!ok[u]) continue;
-                const float pr = exp2f(zt[u][h] - m_new);
+                const float pr = exp2f(zt[u * GT + h] - m_new);
                 l += pr;
                 uint32_t vw[RBL / 4 > 0 ? RBL / 4 : 1];
                 lds_words<RBL>(vw, st + (TBS + u) * RB + lane * RBL);
@@ -658,7 +688,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         if (d == 0) { cm[h] = M; cl[h] = Lsum; }
     }
     // [phase] 8
-    cluster.sync();                                            // CTA partials visible
+    row_sync(cluster, N);                                            // CTA partials visible
 
     // final merge across the cluster; CTA `rank` writes its slice of [G, D]
     {
@@ -668,14 +698,14 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         for (int e = e0 + tid; e < e1; e += kNT) {
             const int h = e / D, d = e - h * D;
             float M = -INFINITY;
-            for (int r = 0; r < N; ++r) M = fmaxf(M, cluster.map_shared_rank(cm, r)[h]);
+            for (int r = 0; r < N; ++r) M = fmaxf(M, row_smem(cluster, N, cm, r)[h]);
             float O = 0.f, Lsum = 0.f;
             for (int r = 0; r < N; ++r) {
-                const float mr = cluster.map_shared_rank(cm, r)[h];
+                const float mr = row_smem(cluster, N, cm, r)[h];
                 if (mr == -INFINITY) continue;
                 const float f = exp2f(mr - M);
-                O = fmaf(f, cluster.map_shared_rank(co, r)[h * D + d], O);
-                Lsum = fmaf(f, cluster.map_shared_rank(cl, r)[h], Lsum);
+                O = fmaf(f, row_smem(cluster, N, co, r)[h * D + d], O);
+                Lsum = fmaf(f, row_smem(cluster, N, cl, r)[h], Lsum);
             }
             const float res = O / Lsum;
             const size_t oidx = (size_t)row * G * D + (size_t)h * D + d;
@@ -684,7 +714,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         }
     }
     // [phase] 9
-    cluster.sync();                                            // keep smem alive for readers
+    row_sync(cluster, N);                                            // keep smem alive for readers
 }
 
 }  // namespace ds

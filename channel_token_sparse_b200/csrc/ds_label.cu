@@ -47,39 +47,10 @@ __global__ void __launch_bounds__(kLabNT) ds_label_kernel(const TKV* __restrict_
             out[e] = rows[t * D + idx_s[j]];
         }
     } else {
-        // 4-bit: one thread per token, fp32 arithmetic with IEEE division and
-        // round-half-even, as stated in include/ds.h
-        for (int t = threadIdx.x; t < nt; t += kLabNT) {
-            const TKV* r = rows + t * D;
-            float mn = E::to_f32(r[idx_s[0]]), mx = mn;
-            for (int j = 1; j < c; ++j) {
-                const float x = E::to_f32(r[idx_s[j]]);
-                mn = fminf(mn, x);
-                mx = fmaxf(mx, x);
-            }
-            const float step = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
-            const uint16_t sh = __half_as_ushort(__float2half_rn(step));
-            const uint16_t zh = __half_as_ushort(__float2half_rn(mn));
-            const float sc = fp16_bits_to_f32(sh);
-            const float z = fp16_bits_to_f32(zh);
-            uint8_t* o = label + (tok0 + t) * (size_t)(c / 2);
-            for (int j = 0; j < c; j += 2) {
-                uint32_t nib[2];
-#pragma unroll
-                for (int e2 = 0; e2 < 2; ++e2) {
-                    uint32_t code = 0;
-                    if (sc > 0.f) {
-                        float qv = rintf(__fdiv_rn(__fsub_rn(E::to_f32(r[idx_s[j + e2]]), z), sc));
-                        qv = fminf(fmaxf(qv, 0.f), 15.f);
-                        code = (uint32_t)qv;
-                    }
-                    nib[e2] = code;
-                }
-                o[j / 2] = (uint8_t)(nib[0] | (nib[1] << 4));
-            }
-            lscale[tok0 + t] = sh;
-            lzero[tok0 + t] = zh;
-        }
+        // 4-bit: one thread per token (pack_int4_row states the arithmetic)
+        for (int t = threadIdx.x; t < nt; t += kLabNT)
+            pack_int4_row<TKV>(rows + t * D, idx_s, c, label + (tok0 + t) * (size_t)(c / 2), lscale + tok0 + t,
+                               lzero + tok0 + t);
     }
 }
 

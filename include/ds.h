@@ -148,6 +148,19 @@ DS_API ds_status ds_sparse_decode(const void* q, const void* k, const void* v, d
                            float sm_scale, void* out, ds_dtype out_dt,
                            int32_t* sel_out, float* score_out, cudaStream_t stream);
 
+/* One decode step in one launch (Double Sparsity 离线校准 + 在线前向计算):
+ * the label row of the newest token, position s-1, whose K/V the caller has
+ * already written, is built exactly as ds_append_label builds it and stored
+ * to label (and lscale/lzero for 4-bit); then the step runs exactly as
+ * ds_sparse_decode over tokens [0, s). Same arguments and rules as
+ * ds_sparse_decode; only row s-1 of the label cache is written. */
+DS_API ds_status ds_decode_step(const void* q, const void* k, const void* v, ds_dtype kvdt,
+                                void* label, ds_dtype label_dt,
+                                uint16_t* lscale, uint16_t* lzero, const int32_t* idx,
+                                int b, int hq, int hkv, int s, int s_cap, int d, int c, int topk,
+                                float sm_scale, void* out, ds_dtype out_dt,
+                                int32_t* sel_out, float* score_out, cudaStream_t stream);
+
 /* Launch plan of ds_sparse_decode for a shape (host only, launches nothing):
  * CTAs per thread-block cluster (one cluster per (b, kv head)), tokens per
  * CTA and dynamic shared memory per CTA in bytes. Any output may be NULL. */

@@ -341,3 +341,54 @@ def _full_config(i, rows_to_check):
 ])
 def test_full_size_configs(i, rows):
     _full_config(i, rows)
+
+
+# ------------------------------------------------------- fused decode step
+
+@pytest.mark.parametrize("kv,label,d,c,hq,hkv,s,topk,cluster", [
+    ("bf16", "bf16", 128, 16, 8, 4, 3001, 200, 0),
+    ("bf16", "bf16", 128, 16, 8, 4, 3001, 200, 4),
+    ("bf16", "int4", 128, 32, 4, 4, 2500, 160, 0),
+    ("bf16", "int4", 128, 32, 4, 4, 2500, 160, 16),
+    ("f32", "f32", 64, 8, 4, 2, 777, 50, 2),
+    ("f32", "int4", 64, 16, 2, 2, 300, 400, 0),   # k >= s: select all
+])
+def test_decode_step_equals_append_then_decode(kv, label, d, c, hq, hkv, s, topk, cluster):
+    """ds_decode_step = ds_append_label(s - 1) + ds_sparse_decode, bit for bit,
+    and it matches the oracle."""
+    wl = synth.custom(b=2, hq=hq, hkv=hkv, d=d, s=s, c=c, topk=topk, kv_dtype=kv, label_dtype=label,
+                      n_outlier=min(16, c), outlier_scale=6.0, index=73)
+    di = synth.decode_inputs(wl, s_cap=s + 5)
+    idx = _idx_random(wl, 7)
+    qd, kd, vd = (to_dev(x, kv) for x in (di.q, di.k, di.v))
+    idxd = torch.from_numpy(idx).cuda()
+    lab1, sc1, ze1 = _gpu_label(kd, idxd, s - 1, wl)      # prefill of s - 1 tokens only
+    lab2, sc2, ze2 = _gpu_label(kd, idxd, s, wl)          # prefill of all s tokens
+    ds.set_cluster(cluster)
+    try:
+        sel1 = torch.full((wl.b, hkv, topk), -7, dtype=torch.int32, device="cuda")
+        sel2 = sel1.clone()
+        s1 = torch.zeros((wl.b, hkv, s), dtype=torch.float32, device="cuda")
+        s2 = s1.clone()
+        o1 = ds.decode_step(qd, kd, vd, lab1, idxd, s, topk, lscale=sc1, lzero=ze1, sel_out=sel1, score_out=s1)
+        o2 = ds.sparse_decode(qd, kd, vd, lab2, idxd, s, topk, lscale=sc2, lzero=ze2, sel_out=sel2, score_out=s2)
+        torch.cuda.synchronize()
+    finally:
+        ds.set_cluster(0)
+    assert torch.equal(lab1, lab2)
+    if sc1 is not None:
+        assert torch.equal(sc1, sc2) and torch.equal(ze1, ze2)
+    assert torch.equal(s1, s2) and torch.equal(sel1, sel2) and torch.equal(o1, o2)
+    ref_label = oracle.build_label(di.k, kv, label, idx, s)
+    got = _host_label(lab1, sc1, ze1, wl)
+    if label == "int4":
+        for a, b_ in zip(got, ref_label):
+            assert np.array_equal(a, b_)
+    else:
+        assert np.array_equal(got, ref_label)
+    _, sel_ref, s_ref = oracle.sparse_decode(di.q, di.k, di.v, kv, ref_label, label, idx, s, topk)
+    check_scores(s1.cpu().numpy(), s_ref)
+    sg = sel1.cpu().numpy()
+    check_selection(sg.reshape(-1, topk), sel_ref.reshape(-1, topk), s_ref.reshape(-1, s), topk, s)
+    o_ref = oracle.attention(di.q, di.k, di.v, kv, sg, hkv)
+    assert np.abs(o1.cpu().numpy() - o_ref).max() <= OUT_ATOL

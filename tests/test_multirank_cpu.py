@@ -62,6 +62,7 @@ def test_algorithmic_bytes_match_hand_count():
     import synth
     ab = bench.algorithmic_bytes(synth.workload(1), out_esz=2)
     assert ab["label"] == 33554432 and ab["kv_selected"] == 33554432 and ab["q_out"] == 131072
-    assert ab["total"] == 67239936
+    assert ab["append"] == 8 * 32 * (256 + 32)  # new token's key row read + label row written
+    assert ab["total"] == 67239936 + 8 * 32 * 288
     ab2 = bench.algorithmic_bytes(synth.workload(2), out_esz=2)
     assert ab2["label"] == 32 * 32 * 16384 * 20  # 16 B payload + fp16 scale + fp16 zero
