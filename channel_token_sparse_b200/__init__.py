@@ -31,6 +31,7 @@ SIGNATURES = {
     "ds_last_error": (C.c_char_p, []),
     "ds_calibrate_workspace_size": (_i, [_i, _i, _i, _i, _i, _i, C.POINTER(_sz)]),
     "ds_calibrate_channels": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp]),
+    "ds_calibrate_channels_noalloc": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
     "ds_build_label_cache": (_i, [_vp, _i, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _vp]),
     "ds_append_label": (_i, [_vp, _i, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _vp]),
     "ds_sparse_decode": (_i, [_vp, _vp, _vp, _i, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
@@ -157,6 +158,18 @@ def calibrate_channels(q_win, k, c: int, ratio_out=None, idx_out=None, ws=None, 
     _check(lib().ds_calibrate_channels(_ptr(q_win), _ptr(k), _kv_dtype(k), n, hq, hkv, w, s, d, c,
                                        _ptr(ratio_out), _ptr(idx_out), _ptr(ws), ws.numel(),
                                        _stream(stream)))
+    return idx_out, ratio_out
+
+
+def calibrate_channels_noalloc(q_win, k, c: int, ratio_out, idx_out, stream=None):
+    """ds_calibrate_channels with the library's fixed scratch instead of a
+    workspace (for callers that cannot allocate device memory); the outputs
+    must be provided."""
+    _need_cuda(q_win, k, ratio_out, idx_out)
+    n, hq, w, d = q_win.shape
+    _, hkv, s, _ = k.shape
+    _check(lib().ds_calibrate_channels_noalloc(_ptr(q_win), _ptr(k), _kv_dtype(k), n, hq, hkv, w, s, d, c,
+                                               _ptr(ratio_out), _ptr(idx_out), _stream(stream)))
     return idx_out, ratio_out
 
 

@@ -232,6 +232,29 @@ ds_status ds_calibrate_channels(const void* q_win, const void* k, ds_dtype dt, i
     return DS_OK;
 }
 
+ds_status ds_calibrate_channels_noalloc(const void* q_win, const void* k, ds_dtype dt, int n_samples,
+                                        int hq, int hkv, int w, int s, int d, int c, float* ratio_out,
+                                        int32_t* idx_out, cudaStream_t stream) {
+    size_t need = 0;
+    ds_status r = ds_calibrate_workspace_size(n_samples, hq, hkv, w, s, d, &need);
+    if (r != DS_OK) return r;
+    if (!kv_dtype_ok(dt)) return fail(DS_ERR_UNSUPPORTED, "dtype %d (supported: f32, bf16)", (int)dt);
+    if (c < 1 || c > d) return fail(DS_ERR_INVALID_ARG, "need 1 <= c (%d) <= d (%d)", c, d);
+    if (hq / hkv * (long long)w > (1 << 20)) return fail(DS_ERR_UNSUPPORTED, "window too large");
+    if (!q_win || !k || !idx_out) return fail(DS_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(q_win) || !aligned16(k) || !aligned16(idx_out) || (ratio_out && !aligned16(ratio_out)))
+        return fail(DS_ERR_INVALID_ARG, "pointer not 16-byte aligned");
+    const size_t cap = ds::calib_static_scratch_bytes();
+    if (need > cap)
+        return fail(DS_ERR_WORKSPACE,
+                    "calibration needs %zu B of scratch (n_samples * hkv * (2d + 1) doubles); the fixed "
+                    "scratch holds %zu B: use ds_calibrate_channels with a workspace", need, cap);
+    ds::CalibArgs a{q_win, k, dt == DS_BF16, n_samples, hq, hkv, w, s, d, c, ratio_out, idx_out, nullptr};
+    cudaError_t e = ds::launch_calib_static(a, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "calibration launch (fixed scratch)");
+    return DS_OK;
+}
+
 ds_status ds_build_label_cache(const void* k, ds_dtype kdt, const int32_t* idx, int b, int hkv,
                                int s, int s_cap, int d, int c, void* label, ds_dtype label_dt,
                                uint16_t* lscale, uint16_t* lzero, cudaStream_t stream) {

@@ -11,6 +11,8 @@
 // entries of Q K^T (fp32 dot products, fp64 accumulation) into the caller's
 // workspace, then one CTA per kv head forms r (mean over samples) and ranks
 // the channels (ties to the lower channel index).
+#include <mutex>
+
 #include "ds_common.cuh"
 #include "ds_internal.h"
 
@@ -146,6 +148,58 @@ cudaError_t launch_calib(const CalibArgs& a, cudaStream_t st) {
         if (a.d == 128) return launch_calib_t<float, 128>(a, st);
     }
     return cudaErrorInvalidValue;
+}
+
+}  // namespace ds
+
+// ------------------------------------------------ calibration without allocation
+//
+// For callers that cannot obtain device memory from cudaMalloc or a caching
+// allocator: code running while a CUDA graph is being captured, hosts that
+// hand a plugin only fixed tensors and own every allocation, or runtimes with
+// a preallocated device budget. The scratch then lives in this fixed
+// file-scope array, which every GPU that loads the library keeps until exit.
+// All calls share it and each call first clears the part it uses; calls that
+// overlap on the GPU (different streams, no ordering between them) race on it.
+namespace {
+
+constexpr size_t kStaticCalibDoubles = 131072;  // 1 MiB
+static __device__ __align__(256) double g_calib_static_scratch[kStaticCalibDoubles];
+
+std::mutex g_static_mu;
+void* g_static_ptr[64] = {};  // device address of the array, per device ordinal
+
+// Device address of the scratch array on the current device. Host code sees
+// the array's name as a host-side stand-in, so the address is looked up once
+// per device (with that device current) and cached.
+cudaError_t static_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_static_mu);
+    if (!g_static_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_calib_static_scratch);
+        if (e != cudaSuccess) return e;
+        g_static_ptr[dev] = p;
+    }
+    *out = g_static_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+namespace ds {
+
+size_t calib_static_scratch_bytes() { return kStaticCalibDoubles * sizeof(double); }
+
+cudaError_t launch_calib_static(CalibArgs a, cudaStream_t st) {
+    void* p = nullptr;
+    const cudaError_t e = static_scratch(&p);
+    if (e != cudaSuccess) return e;
+    a.ws = p;
+    return launch_calib(a, st);
 }
 
 }  // namespace ds

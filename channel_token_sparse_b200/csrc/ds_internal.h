@@ -39,5 +39,8 @@ struct CalibArgs {
 };
 size_t calib_workspace_bytes(int n, int hkv, int d);
 cudaError_t launch_calib(const CalibArgs& a, cudaStream_t st);
+// Same launch with the scratch taken from a fixed device array (no allocation).
+size_t calib_static_scratch_bytes();
+cudaError_t launch_calib_static(CalibArgs a, cudaStream_t st);
 
 }  // namespace ds

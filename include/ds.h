@@ -98,6 +98,25 @@ DS_API ds_status ds_calibrate_channels(const void* q_win, const void* k, ds_dtyp
                                 float* ratio_out, int32_t* idx_out,
                                 void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* Calibration for callers that cannot allocate device memory -- code that
+ * runs while a CUDA graph is being captured, plugins whose host framework owns
+ * every allocation, or runtimes with a fixed device budget. It has no
+ * counterpart on the pages; it computes exactly what ds_calibrate_channels
+ * computes, with the same arguments minus the workspace. Its scratch is a
+ * fixed 1 MiB device array inside the library (held by every GPU that loads
+ * the library until the process exits), so it needs
+ * n_samples * hkv * (2*d + 1) * 8 <= 1048576 bytes (ds_calibrate_workspace_size
+ * gives the figure); larger problems get DS_ERR_WORKSPACE with the numbers.
+ * It allocates nothing and calls no allocating routine. The first call on a
+ * device looks up the array's device address (once per device, with that
+ * device current); make that first call before any stream capture. All calls
+ * share the array and each clears the part it uses: calls that may run
+ * concurrently on the GPU (different streams without ordering) race on it. */
+DS_API ds_status ds_calibrate_channels_noalloc(const void* q_win, const void* k, ds_dtype dt,
+                                               int n_samples, int hq, int hkv, int w, int s, int d,
+                                               int c, float* ratio_out, int32_t* idx_out,
+                                               cudaStream_t stream);
+
 /* ----------------------------------------------------------- label cache
  * Prefill (Double Sparsity 离线校准, label cache paragraph): copy the heavy
  * channels of tokens [0, s) of the key cache into the label cache.
