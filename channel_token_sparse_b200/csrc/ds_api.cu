@@ -62,8 +62,11 @@ constexpr int kMaxSmem = 227 * 1024;
 constexpr int kCtasPerSm = 2;  // __launch_bounds__(256, 2) -> <= 128 registers
 
 struct Plan {
-    int N, chunk, lay_chunk, per, smem;
+    int N, chunk, lay_chunk, per, smem, att_stages, lab_ring;
 };
+
+// Two CTAs of 256 threads per SM: each may use up to (228 KiB - 2 KiB) / 2.
+constexpr int kSmemFor2 = (228 * 1024 - 2 * 1024) / 2;
 
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
@@ -71,12 +74,12 @@ int round_up(int x, int m) { return (x + m - 1) / m * m; }
 // grid (rows * N CTAs) still fits in one wave of resident CTAs, keeping at
 // least 256 tokens per CTA; rows beyond one wave use N = 1. A forced N
 // (ds_sparse_decode_set_cluster) overrides the choice when feasible.
-bool make_plan(int rows, int G, int s, int d, int c, int topk, bool dense, int esz, int slots,
+bool make_plan(int rows, int G, int s, int d, int c, int topk, bool dense, bool int4, int esz, int slots,
                int forced, Plan* out) {
     const int GT = group_tier(G);
     const bool select_all = dense || topk >= s;
     const int k_eff = topk < s ? topk : s;
-    Plan best{0, 0, 0, 0, 0};
+    Plan best{0, 0, 0, 0, 0, 0, 0};
     for (int N = 1; N <= 16; N *= 2) {
         Plan p;
         p.N = N;
@@ -84,8 +87,22 @@ bool make_plan(int rows, int G, int s, int d, int c, int topk, bool dense, int e
         if (p.chunk > ds::kMaxChunk) continue;
         p.lay_chunk = dense ? 0 : p.chunk;
         p.per = select_all ? 0 : (k_eff + N - 1) / N;
-        p.smem = ds::decode_smem_layout(GT, d, c, p.lay_chunk, p.per, esz).total;
+        // bf16 K/V: 3 attention stages per warp when two CTAs still fit per SM, else 2
+        p.att_stages = esz == 2 ? 3 : ds::kAttStagesF32;
+        p.smem = ds::decode_smem_layout(GT, d, c, p.lay_chunk, p.per, esz, p.att_stages).total;
+        if (esz == 2 && p.smem > kSmemFor2) {
+            p.att_stages = 2;
+            p.smem = ds::decode_smem_layout(GT, d, c, p.lay_chunk, p.per, esz, p.att_stages).total;
+        }
         if (p.smem > kMaxSmem) continue;
+        // fp labels of 16-byte multiples stream through a shared-memory ring
+        // placed behind the 16-bit keys when the region has room for it
+        p.lab_ring = 0;
+        if (!dense && !int4 && (c * esz) % 16 == 0) {
+            const ds::DecodeSmem L = ds::decode_smem_layout(GT, d, c, p.lay_chunk, p.per, esz, p.att_stages);
+            const int region = L.total - L.region;
+            if (ds::align16(p.lay_chunk * 2) + ds::lab_ring_bytes(c * esz) <= region) p.lab_ring = 1;
+        }
         if (forced) {
             if (N == forced) { *out = p; return true; }
             continue;
@@ -277,7 +294,8 @@ ds_status ds_sparse_decode_plan(int b, int hq, int hkv, int s, int d, int c, int
     if (label_dt != DS_INT4 && label_dt != kvdt) return fail(DS_ERR_INVALID_ARG, "label dtype");
     if (topk < 1) return fail(DS_ERR_INVALID_ARG, "topk must be >= 1");
     Plan pl;
-    if (!make_plan(b * hkv, hq / hkv, s, d, c, topk, false, kvdt == DS_F32 ? 4 : 2, kCtasPerSm * 148,
+    if (!make_plan(b * hkv, hq / hkv, s, d, c, topk, false, label_dt == DS_INT4, kvdt == DS_F32 ? 4 : 2,
+                   kCtasPerSm * 148,
                    g_cluster_override.load(), &pl))
         return fail(DS_ERR_UNSUPPORTED, "no feasible launch plan (s too long for 16 CTAs per row)");
     if (cluster_out) *cluster_out = pl.N;
@@ -309,7 +327,8 @@ ds_status sparse_decode_impl(const void* q, const void* k, const void* v, ds_dty
     const int G = hq / hkv, GT = group_tier(G);
     const int rows = b * hkv;
     Plan pl;
-    if (!make_plan(rows, G, s, d, c, topk, false, kvdt == DS_F32 ? 4 : 2, kCtasPerSm * sm_count(),
+    if (!make_plan(rows, G, s, d, c, topk, false, label_dt == DS_INT4, kvdt == DS_F32 ? 4 : 2,
+                   kCtasPerSm * sm_count(),
                    g_cluster_override.load(), &pl))
         return fail(DS_ERR_UNSUPPORTED, "no feasible launch plan (s too long for 16 CTAs per row)");
     ds::DecodeKernel kern = pick_kernel(kvdt, label_dt == DS_INT4, d, c, GT);
@@ -320,6 +339,8 @@ ds_status sparse_decode_impl(const void* q, const void* k, const void* v, ds_dty
     p.hkv = hkv; p.G = G; p.s = s; p.s_cap = s_cap; p.topk = topk;
     p.chunk = pl.chunk; p.lay_chunk = pl.lay_chunk; p.per = pl.per;
     p.append = append ? 1 : 0;
+    p.att_stages = pl.att_stages;
+    p.lab_ring = pl.lab_ring;
     const float scale = sm_scale > 0.f ? sm_scale : 1.0f / sqrtf((float)d);
     p.qscale = scale * 1.4426950408889634f;
     p.out_bf16 = out_dt == DS_BF16;
@@ -362,7 +383,7 @@ ds_status ds_dense_decode(const void* q, const void* k, const void* v, ds_dtype 
     const int G = hq / hkv, GT = group_tier(G);
     const int rows = b * hkv;
     Plan pl;
-    if (!make_plan(rows, G, s, d, 8, s, true, kvdt == DS_F32 ? 4 : 2, kCtasPerSm * sm_count(),
+    if (!make_plan(rows, G, s, d, 8, s, true, false, kvdt == DS_F32 ? 4 : 2, kCtasPerSm * sm_count(),
                    g_cluster_override.load(), &pl))
         return fail(DS_ERR_UNSUPPORTED, "no feasible launch plan");
     ds::DecodeKernel kern = pick_kernel(kvdt, false, d, 8, GT);
@@ -371,6 +392,8 @@ ds_status ds_dense_decode(const void* q, const void* k, const void* v, ds_dtype 
     p.q = q; p.k = k; p.v = v; p.out = out;
     p.hkv = hkv; p.G = G; p.s = s; p.s_cap = s_cap; p.topk = s;
     p.chunk = pl.chunk; p.lay_chunk = 0; p.per = 0;
+    p.att_stages = pl.att_stages;
+    p.lab_ring = pl.lab_ring;
     const float scale = sm_scale > 0.f ? sm_scale : 1.0f / sqrtf((float)d);
     p.qscale = scale * 1.4426950408889634f;
     p.out_bf16 = out_dt == DS_BF16;

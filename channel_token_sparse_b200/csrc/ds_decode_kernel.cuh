@@ -54,6 +54,8 @@ struct DecodeParams {
     int lay_chunk; // chunk used to size shared memory (0 in dense mode)
     int per;       // selected tokens attended per CTA (ceil(min(topk,s) / N))
     int append;    // 1: first build the label row of token s-1 from the key cache (decode step)
+    int att_stages; // attention ring stages per warp (bf16: 2 or 3; fp32: kAttStagesF32)
+    int lab_ring;  // 1: fp label rows stream through a shared-memory ring behind the keys
     float qscale;  // sm_scale * log2(e)
     int out_bf16;
     int dense;     // 1: attend every token, no label / scores / selection
@@ -61,31 +63,37 @@ struct DecodeParams {
 
 // Shared-memory carve-up (bytes), identical on host and device.
 struct DecodeSmem {
-    int qs, qL, idx, histA, histB, ctl, scan, cm, cl, co, bits, blist, app, sel, region, total;
+    int qs, qa, qL, idx, histA, histB, ctl, scan, cm, cl, co, bits, blist, app, sel, region, total;
 };
 
 __host__ __device__ inline int align16(int x) { return (x + 15) & ~15; }
 
-// Attention-phase staging: each warp owns a ring of kAttStages stages; a
-// stage holds the K rows then the V rows of att_stage_tokens(row bytes)
-// tokens (~2 KiB per stage). A warp's partial softmax state (at most
-// 8 * (128 + 2) floats) is later written into its own ring.
-constexpr int kAttStages = 4;
+// Attention-phase staging: each warp owns a ring of shared-memory stages; a
+// stage holds the K rows then the V rows of att_stage_tokens() tokens. With
+// bf16 K/V a stage is 8 tokens (one 8-token tensor-core tile; 2 or 3 stages,
+// chosen by the host from the shared-memory budget); with fp32 K/V, ~1 KiB
+// of rows per stage and kAttStagesF32 stages. A warp's partial softmax state
+// (at most 8 * (128 + 2) floats) is later written into its own ring.
+constexpr int kAttStagesF32 = 4;
+// Label-streaming ring (fp labels): stages of one row per thread.
+constexpr int kLabStages = 6;
+__host__ __device__ constexpr int lab_ring_bytes(int label_row_bytes) { return kLabStages * 256 * label_row_bytes; }
+__host__ __device__ constexpr int att_stage_tokens(int row_bytes, int elem_bytes) {
+    return elem_bytes == 2 ? 8 : (row_bytes >= 1024 ? 1 : 1024 / row_bytes);
+}
+__host__ __device__ constexpr int att_ring_bytes(int row_bytes, int elem_bytes, int stages) {
+    return stages * att_stage_tokens(row_bytes, elem_bytes) * 2 * row_bytes;
+}
 // Tokens of the k-th key's 16-bit bucket kept in a list for the last radix
 // pass (a CTA whose bucket is larger falls back to sweeping its keys).
 constexpr int kBucketCap = 1024;
-__host__ __device__ constexpr int att_stage_tokens(int row_bytes) {
-    return row_bytes >= 1024 ? 1 : 1024 / row_bytes;
-}
-__host__ __device__ constexpr int att_ring_bytes(int row_bytes) {
-    return kAttStages * att_stage_tokens(row_bytes) * 2 * row_bytes;
-}
 
 __host__ __device__ inline DecodeSmem decode_smem_layout(int GT, int D, int C, int chunk, int per,
-                                                         int elem_bytes) {
+                                                         int elem_bytes, int att_stages) {
     DecodeSmem L;
     int o = 0;
     L.qs = o;     o += align16(GT * D * 4);
+    L.qa = o;     o += elem_bytes == 2 ? (D / 16) * 32 * 8 : 0;  // packed bf16 Q fragments
     L.qL = o;     o += align16(C * 4);
     L.idx = o;    o += align16(C * 4);
     L.histA = o;  o += 256 * 4;
@@ -101,7 +109,7 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int GT, int D, int C, i
     L.sel = o;    o += align16(per * 4);
     L.region = o;
     const int keys = chunk * 2;
-    const int ring = kNW * att_ring_bytes(D * elem_bytes);
+    const int ring = kNW * att_ring_bytes(D * elem_bytes, elem_bytes, att_stages);
     o += align16(keys > ring ? keys : ring);
     L.total = o;
     return L;
@@ -210,7 +218,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     const int tid = threadIdx.x, lane = lane_id(), wid = warp_id();
 
     extern __shared__ __align__(16) uint8_t smem[];
-    const DecodeSmem L = decode_smem_layout(GT, D, C, p.lay_chunk, p.per, E::kBytes);
+    const DecodeSmem L = decode_smem_layout(GT, D, C, p.lay_chunk, p.per, E::kBytes, p.att_stages);
     float* qs = reinterpret_cast<float*>(smem + L.qs);
     float* qLs = reinterpret_cast<float*>(smem + L.qL);
     int* idx_s = reinterpret_cast<int*>(smem + L.idx);
@@ -256,6 +264,15 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
             float a = 0.f;
             for (int e = 0; e < G; ++e) a += qs[e * D + idx_s[j]];
             qLs[j] = a;
+        }
+    }
+    if constexpr (E::kBytes == 2) {
+        // tensor-core A fragments of q for the attention phase (see step 3b)
+        uint2* qa_w = reinterpret_cast<uint2*>(smem + L.qa);
+        for (int e = tid; e < (D / 16) * 32; e += kNT) {
+            const int c = e >> 5, ln = e & 31, h = ln >> 2, col = 16 * c + (ln & 3) * 2;
+            const float* qh = qs + h * D + col;
+            qa_w[e] = h < G ? make_uint2(pack_bf16x2(qh[0], qh[1]), pack_bf16x2(qh[8], qh[9])) : make_uint2(0u, 0u);
         }
     }
     // decode step: the CTA holding token s-1 builds its label row (the same
@@ -321,7 +338,53 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
 
     // [phase] 1
     // ---------------------------------------------------------------- step 2
-    if (need_scores) {
+    // Score one token (local index i) from its label row, store its 16-bit
+    // key and count its top byte.
+    auto score_token = [&](int i, const uint32_t (&w)[LG::kWords], float ss, float zz) {
+        const float sv = label_score<TKV, LK, C>(w, qreg, qLs, ss, zz, qsum);
+        const uint32_t key = score_key(sv);
+        if (!select_all) {
+            keys[i] = (uint16_t)(key >> 16);
+            atomicAdd(&histA[key >> 24], 1u);
+        }
+        if (p.score_out) p.score_out[(size_t)row * s + t0 + i] = sv;
+    };
+    constexpr bool kRingable = LK == kLabelFp && LG::kBytes % 16 == 0;
+    if (kRingable && need_scores && p.lab_ring) {
+        // fp label rows stream through a kLabStages-deep shared-memory ring
+        // with cp.async (no registers held while in flight): in stage j,
+        // thread tid copies and then scores local token j * kNT + tid, so it
+        // only ever reads its own copies (no block barrier needed)
+        uint8_t* lring = smem + L.region + align16(p.lay_chunk * 2);
+        constexpr int kSlot = LG::kBytes;               // bytes per token
+        constexpr int kStage = kNT * kSlot;
+        const int nst = (n_loc + kNT - 1) / kNT;
+        auto issue = [&](int j) {
+            const int i = j * kNT + tid;
+            if (j < nst && i < n_loc && i != app_i) {
+                uint8_t* dst = lring + (j % kLabStages) * kStage + tid * kSlot;
+                const uint8_t* src = lab + (size_t)(t0 + i) * kSlot;
+#pragma unroll
+                for (int o = 0; o < kSlot; o += 16) cp_async16(dst + o, src + o);
+            }
+        };
+#pragma unroll 1
+        for (int j = 0; j < kLabStages - 1; ++j) { issue(j); cp_async_commit(); }
+#pragma unroll 1
+        for (int j = 0; j < nst; ++j) {
+            issue(j + kLabStages - 1);
+            cp_async_commit();
+            cp_async_wait<kLabStages - 1>();
+            const int i = j * kNT + tid;
+            if (i < n_loc) {
+                uint32_t w[LG::kWords];
+                if (i == app_i) lds_row<LG::kBytes>(w, app_row);
+                else lds_row<LG::kBytes>(w, lring + (j % kLabStages) * kStage + tid * kSlot);
+                score_token(i, w, 0.f, 0.f);
+            }
+        }
+        cp_async_wait<0>();
+    } else if (need_scores) {
         for (int base = 0; base < n_loc; base += kRound) {
             uint32_t w[U][LG::kWords];
             float sc[U], z[U];
@@ -333,20 +396,11 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int i = base + u * kNT + tid;
-                const bool valid = i < n_loc;
-                uint32_t bin = 256u;
-                if (valid) {
+                if (i < n_loc) {
                     float zz = 0.f, ss = 0.f;
                     if constexpr (LK == kLabelInt4) { ss = sc[u]; zz = z[u]; }
-                    const float sv = label_score<TKV, LK, C>(w[u], qreg, qLs, ss, zz, qsum);
-                    const uint32_t key = score_key(sv);
-                    if (!select_all) {
-                        keys[i] = (uint16_t)(key >> 16);
-                        bin = key >> 24;
-                    }
-                    if (p.score_out) p.score_out[(size_t)row * s + t0 + i] = sv;
+                    score_token(i, w[u], ss, zz);
                 }
-                if (!select_all && bin < 256u) atomicAdd(&histA[bin], 1u);
             }
         }
     }
@@ -487,9 +541,11 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         }
         // [phase] 16
         // [phase] 17
-        row_sync(cluster, N);                                        // per-CTA counts visible
+        if (N > 1) row_sync(cluster, N);                             // per-CTA counts visible
         // [phase] 18
-        if (wid == 0) {
+        if (N == 1) {
+            if (tid == 0) { ctl[kCtlP] = 0; ctl[kCtlTP] = 0; }
+        } else if (wid == 0) {
             int cs = 0, ct = 0;
             if (lane < N) {
                 const int* rc = row_smem(cluster, N, ctl, lane);
@@ -546,119 +602,236 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
 
     // [phase] 6
     // --------------------------------------------------------------- step 3b
-    // Each warp streams the K and V rows of its tokens through a ring of
-    // kAttStages shared-memory stages with cp.async (16-byte LDGSTS, no
-    // registers held while in flight), kAttStages-1 stages ahead of compute.
-    constexpr int TBS = att_stage_tokens(RB);      // tokens per stage
-    constexpr int kStageBytes = 2 * TBS * RB;
-    constexpr int kPiecesPerRow = RB / 16;
     const int n_att = select_all ? n_loc : max(0, min(p.per, k_eff - rank * p.per));
-    uint8_t* ring = smem + L.region + wid * att_ring_bytes(RB);
-    const int nb = n_att > wid * TBS ? (n_att - wid * TBS + kNW * TBS - 1) / (kNW * TBS) : 0;
     auto att_token = [&](int j) -> int { return select_all ? t0 + j : sel_list[j]; };
-    auto issue_stage = [&](int bi) {
-        const int bt0 = (wid + bi * kNW) * TBS;
-        uint8_t* st = ring + (bi % kAttStages) * kStageBytes;
-        for (int pc = lane; pc < 2 * TBS * kPiecesPerRow; pc += 32) {
-            const int r = pc / kPiecesPerRow, off = (pc - r * kPiecesPerRow) * 16;
-            const int u = r < TBS ? r : r - TBS;
-            if (bt0 + u < n_att) {
-                const TKV* src = (r < TBS ? kb : vb) + (size_t)att_token(bt0 + u) * D;
-                cp_async16(st + r * RB + off, reinterpret_cast<const uint8_t*>(src) + off);
+    float* wp_out = nullptr;  // this warp's partial (m, l, o) per head, [GT][D + 2]
+    if constexpr (E::kBytes == 2) {
+        // bf16 K/V: tensor cores (mma.sync, fp32 accumulate) on 8-token tiles.
+        //   Z  = Q K^T   m16n8k16: rows = the group's heads (padded to 16),
+        //                cols = 8 tokens, k = 16 dims per step
+        //   O^T += V^T P^T  m16n8k8: rows = 16 dims, cols = heads, k = 8 tokens
+        // so the softmax probabilities of a head (a row of Z's accumulator)
+        // are already laid out as the B operand of the second product. P is
+        // split into bf16 hi + lo parts (two products), keeping ~2^-17 of
+        // relative precision. Rows are staged with cp.async into a per-warp
+        // ring; 16-byte chunks are XOR-swizzled by token so that ldmatrix reads
+        // are bank-conflict free.
+        constexpr int TB8 = 8;
+        constexpr int kChunks = RB / 16;           // 16-byte chunks per row
+        constexpr int kStageBytes = 2 * TB8 * RB;
+        const int stages = p.att_stages;
+        uint8_t* ring = smem + L.region + wid * att_ring_bytes(RB, 2, stages);
+        const int nb = n_att > wid * TB8 ? (n_att - wid * TB8 + kNW * TB8 - 1) / (kNW * TB8) : 0;
+        auto issue_stage = [&](int bi) {
+            const int bt0 = (wid + bi * kNW) * TB8;
+            uint8_t* st = ring + (bi % stages) * kStageBytes;
+#pragma unroll
+            for (int pc = lane; pc < 2 * TB8 * kChunks; pc += 32) {
+                const int r = pc / kChunks, c = pc - r * kChunks;
+                const int u = r & (TB8 - 1);
+                const bool ok = bt0 + u < n_att;
+                const TKV* base = r < TB8 ? kb : vb;
+                const TKV* src = ok ? base + (size_t)att_token(bt0 + u) * D : base;
+                // rows of tokens past the end are zero-filled (their p is 0, and 0 * garbage could be NaN)
+                cp_async16_zfill(st + r * RB + ((c ^ u) << 4), reinterpret_cast<const uint8_t*>(src) + (c << 4), ok);
             }
+        };
+        for (int bi = 0; bi < stages - 1; ++bi) {
+            if (bi < nb) issue_stage(bi);
+            cp_async_commit();
         }
-    };
+        // Q fragments (A operand, rows = heads): bf16 pairs, exact (q is bf16),
+        // kept in shared memory ([D/16 steps][32 lanes][2 words]) to spare registers
+        const int hr = lane >> 2, kc = (lane & 3) * 2;
+        const uint2* qa = reinterpret_cast<const uint2*>(smem + L.qa);
+        float o[D / 16][4];
+#pragma unroll
+        for (int i = 0; i < D / 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+        float m_run = -INFINITY, l_run = 0.f;  // for head hr (row of Z)
+        // [phase] 21
 #pragma unroll 1
-    for (int bi = 0; bi < kAttStages - 1; ++bi) {
-        if (bi < nb) issue_stage(bi);
-        cp_async_commit();
-    }
-
-    float qf[GT][EPL];
+        for (int bi = 0; bi < nb; ++bi) {
+            if (bi + stages - 1 < nb) issue_stage(bi + stages - 1);
+            cp_async_commit();
+            if (stages == 3) cp_async_wait<2>();
+            else cp_async_wait<1>();
+            __syncwarp();
+            const uint8_t* st = ring + (bi % stages) * kStageBytes;
+            const int bt0 = (wid + bi * kNW) * TB8;
+            // Z = Q K^T over D in 16-dim steps; one ldmatrix.x4 covers 32 dims
+            float z[4] = {0.f, 0.f, 0.f, 0.f};
+            const int mr = lane & 7, mi = lane >> 3;  // ldmatrix: row (token) and matrix index
 #pragma unroll
-    for (int h = 0; h < GT; ++h)
+            for (int c4 = 0; c4 < D / 32; ++c4) {
+                uint32_t b[4];
+                ldmatrix_x4(b, st + mr * RB + (((4 * c4 + mi) ^ mr) << 4));
+                const uint2 q0 = qa[(2 * c4) * 32 + lane], q1 = qa[(2 * c4 + 1) * 32 + lane];
+                mma_bf16_16816(z, q0.x, 0u, q0.y, 0u, b[0], b[1]);
+                mma_bf16_16816(z, q1.x, 0u, q1.y, 0u, b[2], b[3]);
+            }
+            // online softmax for head hr over tokens kc, kc + 1 of the tile
+            const bool ok0 = bt0 + kc < n_att, ok1 = bt0 + kc + 1 < n_att;
+            const float z0 = ok0 ? z[0] * p.qscale : -INFINITY;
+            const float z1 = ok1 ? z[1] * p.qscale : -INFINITY;
+            float mx = fmaxf(z0, z1);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float m_new = fmaxf(m_run, mx);
+            const float corr = exp2f(m_run - m_new);
+            const float p0 = exp2f(z0 - m_new), p1 = exp2f(z1 - m_new);
+            float rs = p0 + p1;
+            rs += __shfl_xor_sync(0xffffffffu, rs, 1);
+            rs += __shfl_xor_sync(0xffffffffu, rs, 2);
+            l_run = l_run * corr + rs;
+            m_run = m_new;
+            // O^T columns are heads kc, kc + 1: fetch their corrections
+            const float ca = __shfl_sync(0xffffffffu, corr, 4 * kc);
+            const float cb = __shfl_sync(0xffffffffu, corr, 4 * kc + 4);
 #pragma unroll
-        for (int e = 0; e < EPL; ++e)
-            qf[h][e] = h < G ? qs[h * D + lane * EPL + e] * p.qscale : 0.f;
-
-    float m_run[GT], l_run[GT], o_run[GT][EPL];
+            for (int i = 0; i < D / 16; ++i) { o[i][0] *= ca; o[i][1] *= cb; o[i][2] *= ca; o[i][3] *= cb; }
+            const uint32_t ph = pack_bf16x2(p0, p1);
+            const uint32_t pl = pack_bf16x2(p0 - bf16lo(ph), p1 - bf16hi(ph));
+            // O^T += V^T P^T; one ldmatrix.x4.trans covers two 16-dim row tiles
 #pragma unroll
-    for (int h = 0; h < GT; ++h) {
-        m_run[h] = -INFINITY;
-        l_run[h] = 0.f;
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) o_run[h][e] = 0.f;
-    }
-
-    // [phase] 21
-#pragma unroll 1
-    for (int bi = 0; bi < nb; ++bi) {
-        if (bi + kAttStages - 1 < nb) issue_stage(bi + kAttStages - 1);
-        cp_async_commit();
-        cp_async_wait<kAttStages - 1>();
+            for (int m2 = 0; m2 < D / 32; ++m2) {
+                uint32_t a[4];
+                ldmatrix_x4_trans(a, st + (TB8 + mr) * RB + (((4 * m2 + mi) ^ mr) << 4));
+                mma_bf16_1688(o[2 * m2], a[0], a[1], ph);
+                mma_bf16_1688(o[2 * m2], a[0], a[1], pl);
+                mma_bf16_1688(o[2 * m2 + 1], a[2], a[3], ph);
+                mma_bf16_1688(o[2 * m2 + 1], a[2], a[3], pl);
+            }
+            __syncwarp();
+        }
+        cp_async_wait<0>();
         __syncwarp();
-        const uint8_t* st = ring + (bi % kAttStages) * kStageBytes;
-        const int bt0 = (wid + bi * kNW) * TBS;
-        bool ok[TBS];
-        float zt[TBS * GT];  // index u * GT + h
+        // [phase] 7
+        // per-warp partials -> the warp's own ring (its copies have all landed)
+        wp_out = reinterpret_cast<float*>(ring);
 #pragma unroll
-        for (int u = 0; u < TBS; ++u) {
-            ok[u] = bt0 + u < n_att;
-            uint32_t kw[RBL / 4 > 0 ? RBL / 4 : 1];
-            lds_words<RBL>(kw, st + u * RB + lane * RBL);
-            float kf[EPL];
+        for (int i = 0; i < D / 16; ++i) {
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) {
-                if constexpr (E::kBytes == 2) kf[e] = (e & 1) ? bf16hi(kw[e >> 1]) : bf16lo(kw[e >> 1]);
-                else kf[e] = __uint_as_float(kw[e]);
-            }
-#pragma unroll
-            for (int h = 0; h < GT; ++h) {
-                float a = 0.f;
-#pragma unroll
-                for (int e = 0; e < EPL; ++e) a = fmaf(qf[h][e], kf[e], a);
-                zt[u * GT + h] = a;
+            for (int e = 0; e < 4; ++e) {
+                const int h = kc + (e & 1), d = 16 * i + hr + ((e & 2) ? 8 : 0);
+                if (h < G) wp_out[h * (D + 2) + d] = o[i][e];
             }
         }
-        warp_allreduce_n<TBS * GT>(zt);
-#pragma unroll
-        for (int h = 0; h < GT; ++h) {
-            if (h >= G) break;
-            float mx = -INFINITY;
-#pragma unroll
-            for (int u = 0; u < TBS; ++u) if (ok[u]) mx = fmaxf(mx, zt[u * GT + h]);
-            const float m_new = fmaxf(m_run[h], mx);
-            const float corr = exp2f(m_run[h] - m_new);
-            float l = l_run[h] * corr;
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) o_run[h][e] *= corr;
-#pragma unroll
-            for (int u = 0; u < TBS; ++u) {
-                if (!ok[u]) continue;
-                const float pr = exp2f(zt[u * GT + h] - m_new);
-                l += pr;
-                uint32_t vw[RBL / 4 > 0 ? RBL / 4 : 1];
-                lds_words<RBL>(vw, st + (TBS + u) * RB + lane * RBL);
-#pragma unroll
-                for (int e = 0; e < EPL; ++e) {
-                    float vf;
-                    if constexpr (E::kBytes == 2) vf = (e & 1) ? bf16hi(vw[e >> 1]) : bf16lo(vw[e >> 1]);
-                    else vf = __uint_as_float(vw[e]);
-                    o_run[h][e] = fmaf(pr, vf, o_run[h][e]);
+        if ((lane & 3) == 0 && hr < G) { wp_out[hr * (D + 2) + D] = m_run; wp_out[hr * (D + 2) + D + 1] = l_run; }
+    } else {
+        // fp32 K/V: CUDA cores. Each warp streams the K and V rows of its tokens
+        // through a ring of kAttStagesF32 shared-memory stages with cp.async
+        // (16-byte LDGSTS, no registers held while in flight), kAttStagesF32-1
+        // stages ahead of compute; lane l holds dims [l*EPL, l*EPL + EPL).
+        constexpr int kAttStages = kAttStagesF32;
+        constexpr int TBS = att_stage_tokens(RB, E::kBytes);      // tokens per stage
+        constexpr int kStageBytes = 2 * TBS * RB;
+        constexpr int kPiecesPerRow = RB / 16;
+        uint8_t* ring = smem + L.region + wid * att_ring_bytes(RB, E::kBytes, kAttStages);
+        const int nb = n_att > wid * TBS ? (n_att - wid * TBS + kNW * TBS - 1) / (kNW * TBS) : 0;
+        auto issue_stage = [&](int bi) {
+            const int bt0 = (wid + bi * kNW) * TBS;
+            uint8_t* st = ring + (bi % kAttStages) * kStageBytes;
+            for (int pc = lane; pc < 2 * TBS * kPiecesPerRow; pc += 32) {
+                const int r = pc / kPiecesPerRow, off = (pc - r * kPiecesPerRow) * 16;
+                const int u = r < TBS ? r : r - TBS;
+                if (bt0 + u < n_att) {
+                    const TKV* src = (r < TBS ? kb : vb) + (size_t)att_token(bt0 + u) * D;
+                    cp_async16(st + r * RB + off, reinterpret_cast<const uint8_t*>(src) + off);
                 }
             }
-            m_run[h] = m_new;
-            l_run[h] = l;
+        };
+#pragma unroll 1
+        for (int bi = 0; bi < kAttStages - 1; ++bi) {
+            if (bi < nb) issue_stage(bi);
+            cp_async_commit();
         }
-        __syncwarp();
-    }
-    cp_async_wait<0>();
-    __syncwarp();
 
-    // [phase] 7
-    // per-warp partials -> the warp's own ring (its copies have all landed)
-    {
-        float* wp = reinterpret_cast<float*>(ring);
+        float qf[GT][EPL];
+#pragma unroll
+        for (int h = 0; h < GT; ++h)
+#pragma unroll
+            for (int e = 0; e < EPL; ++e)
+                qf[h][e] = h < G ? qs[h * D + lane * EPL + e] * p.qscale : 0.f;
+
+        float m_run[GT], l_run[GT], o_run[GT][EPL];  // per query head of the group
+#pragma unroll
+        for (int h = 0; h < GT; ++h) {
+            m_run[h] = -INFINITY;
+            l_run[h] = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) o_run[h][e] = 0.f;
+        }
+
+        // [phase] 21
+#pragma unroll 1
+        for (int bi = 0; bi < nb; ++bi) {
+            if (bi + kAttStages - 1 < nb) issue_stage(bi + kAttStages - 1);
+            cp_async_commit();
+            cp_async_wait<kAttStages - 1>();
+            __syncwarp();
+            const uint8_t* st = ring + (bi % kAttStages) * kStageBytes;
+            const int bt0 = (wid + bi * kNW) * TBS;
+            bool ok[TBS];
+            float zt[TBS * GT];  // index u * GT + h
+#pragma unroll
+            for (int u = 0; u < TBS; ++u) {
+                ok[u] = bt0 + u < n_att;
+                uint32_t kw[RBL / 4 > 0 ? RBL / 4 : 1];
+                lds_words<RBL>(kw, st + u * RB + lane * RBL);
+                float kf[EPL];
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) {
+                    if constexpr (E::kBytes == 2) kf[e] = (e & 1) ? bf16hi(kw[e >> 1]) : bf16lo(kw[e >> 1]);
+                    else kf[e] = __uint_as_float(kw[e]);
+                }
+#pragma unroll
+                for (int h = 0; h < GT; ++h) {
+                    float a = 0.f;
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) a = fmaf(qf[h][e], kf[e], a);
+                    zt[u * GT + h] = a;
+                }
+            }
+            warp_allreduce_n<TBS * GT>(zt);
+#pragma unroll
+            for (int h = 0; h < GT; ++h) {
+                if (h >= G) break;
+                float mx = -INFINITY;
+#pragma unroll
+                for (int u = 0; u < TBS; ++u) if (ok[u]) mx = fmaxf(mx, zt[u * GT + h]);
+                const float m_new = fmaxf(m_run[h], mx);
+                const float corr = exp2f(m_run[h] - m_new);
+                float l = l_run[h] * corr;
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) o_run[h][e] *= corr;
+#pragma unroll
+                for (int u = 0; u < TBS; ++u) {
+                    if (!ok[u]) continue;
+                    const float pr = exp2f(zt[u * GT + h] - m_new);
+                    l += pr;
+                    uint32_t vw[RBL / 4 > 0 ? RBL / 4 : 1];
+                    lds_words<RBL>(vw, st + (TBS + u) * RB + lane * RBL);
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) {
+                        float vf;
+                        if constexpr (E::kBytes == 2) vf = (e & 1) ? bf16hi(vw[e >> 1]) : bf16lo(vw[e >> 1]);
+                        else vf = __uint_as_float(vw[e]);
+                        o_run[h][e] = fmaf(pr, vf, o_run[h][e]);
+                    }
+                }
+                m_run[h] = m_new;
+                l_run[h] = l;
+            }
+            __syncwarp();
+        }
+        cp_async_wait<0>();
+        __syncwarp();
+
+        // [phase] 7
+        // per-warp partials -> the warp's own ring (its copies have all landed)
+        wp_out = reinterpret_cast<float*>(ring);
+        {
+        float* wp = wp_out;
 #pragma unroll
         for (int h = 0; h < GT; ++h) {
             if (h >= G) break;
@@ -667,12 +840,14 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
             if (lane == 0) { wp[h * (D + 2) + D] = m_run[h]; wp[h * (D + 2) + D + 1] = l_run[h]; }
         }
     }
+    }
     __syncthreads();
     for (int e = tid; e < G * D; e += kNT) {
         const int h = e / D, d = e - h * D;
         float M = -INFINITY;
         auto wpart = [&](int w) -> const float* {
-            return reinterpret_cast<const float*>(smem + L.region + w * att_ring_bytes(RB)) + h * (D + 2);
+            return reinterpret_cast<const float*>(smem + L.region + w * att_ring_bytes(RB, E::kBytes, p.att_stages)) +
+                   h * (D + 2);
         };
         for (int w = 0; w < kNW; ++w) M = fmaxf(M, wpart(w)[D]);
         float O = 0.f, Lsum = 0.f;
