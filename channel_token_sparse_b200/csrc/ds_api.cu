@@ -62,7 +62,7 @@ constexpr int kMaxSmem = 227 * 1024;
 constexpr int kCtasPerSm = 2;  // __launch_bounds__(256, 2) -> <= 128 registers
 
 struct Plan {
-    int N, chunk, lay_chunk, per, smem, att_stages, lab_ring;
+    int N, chunk, lay_chunk, per, smem, att_stages, lab_ring, keep_low;
 };
 
 // Two CTAs of 256 threads per SM: each may use up to (228 KiB - 2 KiB) / 2.
@@ -79,7 +79,7 @@ bool make_plan(int rows, int G, int s, int d, int c, int topk, bool dense, bool 
     const int GT = group_tier(G);
     const bool select_all = dense || topk >= s;
     const int k_eff = topk < s ? topk : s;
-    Plan best{0, 0, 0, 0, 0, 0, 0};
+    Plan best{0, 0, 0, 0, 0, 0, 0, 0};
     for (int N = 1; N <= 16; N *= 2) {
         Plan p;
         p.N = N;
@@ -97,11 +97,22 @@ bool make_plan(int rows, int G, int s, int d, int c, int topk, bool dense, bool 
         if (p.smem > kMaxSmem) continue;
         // fp labels of 16-byte multiples stream through a shared-memory ring
         // placed behind the 16-bit keys when the region has room for it
+        // and the low 16 key bits are kept beside the high ones when they fit too
         p.lab_ring = 0;
-        if (!dense && !int4 && (c * esz) % 16 == 0) {
+        p.keep_low = 0;
+        if (!dense) {
             const ds::DecodeSmem L = ds::decode_smem_layout(GT, d, c, p.lay_chunk, p.per, esz, p.att_stages);
             const int region = L.total - L.region;
-            if (ds::align16(p.lay_chunk * 2) + ds::lab_ring_bytes(c * esz) <= region) p.lab_ring = 1;
+            const int keys = ds::align16(p.lay_chunk * 2);
+            const int ring = (!int4 && (c * esz) % 16 == 0) ? ds::lab_ring_bytes(c * esz) : -1;
+            if (ring >= 0 && 2 * keys + ring <= region) {
+                p.lab_ring = 1;
+                p.keep_low = 1;
+            } else if (ring >= 0 && keys + ring <= region) {
+                p.lab_ring = 1;
+            } else if (2 * keys <= region) {
+                p.keep_low = 1;
+            }
         }
         if (forced) {
             if (N == forced) { *out = p; return true; }
@@ -341,6 +352,7 @@ ds_status sparse_decode_impl(const void* q, const void* k, const void* v, ds_dty
     p.append = append ? 1 : 0;
     p.att_stages = pl.att_stages;
     p.lab_ring = pl.lab_ring;
+    p.keep_low = pl.keep_low;
     const float scale = sm_scale > 0.f ? sm_scale : 1.0f / sqrtf((float)d);
     p.qscale = scale * 1.4426950408889634f;
     p.out_bf16 = out_dt == DS_BF16;
@@ -394,6 +406,7 @@ ds_status ds_dense_decode(const void* q, const void* k, const void* v, ds_dtype 
     p.chunk = pl.chunk; p.lay_chunk = 0; p.per = 0;
     p.att_stages = pl.att_stages;
     p.lab_ring = pl.lab_ring;
+    p.keep_low = pl.keep_low;
     const float scale = sm_scale > 0.f ? sm_scale : 1.0f / sqrtf((float)d);
     p.qscale = scale * 1.4426950408889634f;
     p.out_bf16 = out_dt == DS_BF16;

@@ -56,6 +56,7 @@ struct DecodeParams {
     int append;    // 1: first build the label row of token s-1 from the key cache (decode step)
     int att_stages; // attention ring stages per warp (bf16: 2 or 3; fp32: kAttStagesF32)
     int lab_ring;  // 1: fp label rows stream through a shared-memory ring behind the keys
+    int keep_low;  // 1: the low 16 key bits are kept in shared memory too (no re-scoring)
     float qscale;  // sm_scale * log2(e)
     int out_bf16;
     int dense;     // 1: attend every token, no label / scores / selection
@@ -63,7 +64,7 @@ struct DecodeParams {
 
 // Shared-memory carve-up (bytes), identical on host and device.
 struct DecodeSmem {
-    int qs, qa, qL, idx, histA, histB, ctl, scan, cm, cl, co, bits, blist, app, sel, region, total;
+    int qs, qa, qL, idx, histA, histB, ctl, scan, cm, cl, co, bits, mcache, blist, app, sel, region, total;
 };
 
 __host__ __device__ inline int align16(int x) { return (x + 15) & ~15; }
@@ -104,6 +105,7 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int GT, int D, int C, i
     L.cl = o;     o += align16(GT * 4);
     L.co = o;     o += align16(GT * D * 4);
     L.bits = o;   o += align16(chunk / 8);
+    L.mcache = o; o += align16(chunk / 8 * 2);  // per key group: selected / tie masks
     L.blist = o;  o += chunk > 0 ? kBucketCap * 4 : 0;
     L.app = o;    o += align16(C * 4) + 16;  // appended token's label row (+ fp16 scale, zero)
     L.sel = o;    o += align16(per * 4);
@@ -230,6 +232,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     float* cl = reinterpret_cast<float*>(smem + L.cl);
     float* co = reinterpret_cast<float*>(smem + L.co);
     uint8_t* bits8 = smem + L.bits;                     // bucket flags, one byte per 8 tokens
+    uint16_t* mcache = reinterpret_cast<uint16_t*>(smem + L.mcache);
     uint32_t* blist = reinterpret_cast<uint32_t*>(smem + L.blist);
     int* sel_list = reinterpret_cast<int*>(smem + L.sel);
     uint16_t* keys = reinterpret_cast<uint16_t*>(smem + L.region);
@@ -250,10 +253,60 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     constexpr int U = LG::kU;
     constexpr int kRound = kNT * U;  // tokens per scoring round
 
+    const int app_i = (p.append && !p.dense && s - 1 >= t0 && s - 1 < t0 + n_loc) ? s - 1 - t0 : -1;
+
     // ---------------------------------------------------------- setup, step 1
-    for (int e = tid; e < G * D; e += kNT) qs[e] = E::to_f32(qrow[e]);
+    // The independent global loads go out first -- q, the channel indices and
+    // (decode step) the newest token's key row -- then the label stream's
+    // first copies; the loads are consumed afterwards, so the set-up costs a
+    // single memory round trip.
+    constexpr int kQPer = (GT * D + kNT - 1) / kNT;
+    float qv[kQPer];
+#pragma unroll
+    for (int e = 0; e < kQPer; ++e) {
+        const int x = tid + kNT * e;
+        qv[e] = x < G * D ? E::to_f32(qrow[x]) : 0.f;
+    }
+    const int iv = (!p.dense && tid < C) ? p.idx[(size_t)g * C + tid] : 0;
+    constexpr int kKRowVecs = D * E::kBytes / 16;   // 16-byte pieces of a key row
+    uint4 kv_app = make_uint4(0u, 0u, 0u, 0u);
+    if (app_i >= 0 && tid < kKRowVecs)
+        kv_app = ldg_stream16(reinterpret_cast<const uint8_t*>(p.k) + ((row_tok + (size_t)(s - 1)) * D) * E::kBytes +
+                              tid * 16);
+
+    // fp label rows stream through a kLabStages-deep shared-memory ring with
+    // cp.async (no registers held while in flight): in stage j, thread tid
+    // copies and then scores local token j * kNT + tid, so it only ever reads
+    // its own copies (no block barrier needed).
+    constexpr bool kRingable = LK == kLabelFp && LG::kBytes % 16 == 0;
+    const bool use_ring = kRingable && need_scores && p.lab_ring;
+    uint16_t* low16 = reinterpret_cast<uint16_t*>(smem + L.region + align16(p.lay_chunk * 2));
+    uint8_t* lring = smem + L.region + align16(p.lay_chunk * 2) * (p.keep_low ? 2 : 1);
+    constexpr int kSlot = LG::kBytes;               // bytes per token
+    constexpr int kStage = kNT * kSlot;
+    const int nst = (n_loc + kNT - 1) / kNT;
+    auto issue = [&](int j) {
+        const int i = j * kNT + tid;
+        if (j < nst && i < n_loc && i != app_i) {
+            uint8_t* dst = lring + (j % kLabStages) * kStage + tid * kSlot;
+            const uint8_t* src = lab + (size_t)(t0 + i) * kSlot;
+#pragma unroll
+            for (int o = 0; o < kSlot; o += 16) cp_async16(dst + o, src + o);
+        }
+    };
+    if (use_ring) {
+#pragma unroll 1
+        for (int j = 0; j < kLabStages - 1; ++j) { issue(j); cp_async_commit(); }
+    }
+
+#pragma unroll
+    for (int e = 0; e < kQPer; ++e)
+        if (tid + kNT * e < G * D) qs[tid + kNT * e] = qv[e];
+    // the newest token's key row is staged in `co` (unused until the end)
+    uint8_t* krow_s = reinterpret_cast<uint8_t*>(co);
+    if (app_i >= 0 && tid < kKRowVecs) reinterpret_cast<uint4*>(krow_s)[tid] = kv_app;
     if (!p.dense) {
-        for (int j = tid; j < C; j += kNT) idx_s[j] = min(max(p.idx[(size_t)g * C + j], 0), D - 1);
+        if (tid < C) idx_s[tid] = min(max(iv, 0), D - 1);
         histA[tid] = 0u;
         histB[tid] = 0u;
         if (tid == 0) ctl[kCtlBL] = 0;
@@ -278,9 +331,8 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     // decode step: the CTA holding token s-1 builds its label row (the same
     // copy / 4-bit pack as ds_append_label), keeps it in shared memory and
     // stores it to the label cache
-    const int app_i = (p.append && !p.dense && s - 1 >= t0 && s - 1 < t0 + n_loc) ? s - 1 - t0 : -1;
     if (app_i >= 0 && wid == 0) {
-        const TKV* krow = reinterpret_cast<const TKV*>(p.k) + (row_tok + (size_t)(s - 1)) * D;
+        const TKV* krow = reinterpret_cast<const TKV*>(krow_s);
         uint8_t* grow = const_cast<uint8_t*>(lab) + (size_t)(s - 1) * LG::kBytes;
         if constexpr (LK == kLabelFp) {
             TKV* srow = reinterpret_cast<TKV*>(smem + L.app);
@@ -345,31 +397,12 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         const uint32_t key = score_key(sv);
         if (!select_all) {
             keys[i] = (uint16_t)(key >> 16);
+            if (p.keep_low) low16[i] = (uint16_t)key;
             atomicAdd(&histA[key >> 24], 1u);
         }
         if (p.score_out) p.score_out[(size_t)row * s + t0 + i] = sv;
     };
-    constexpr bool kRingable = LK == kLabelFp && LG::kBytes % 16 == 0;
-    if (kRingable && need_scores && p.lab_ring) {
-        // fp label rows stream through a kLabStages-deep shared-memory ring
-        // with cp.async (no registers held while in flight): in stage j,
-        // thread tid copies and then scores local token j * kNT + tid, so it
-        // only ever reads its own copies (no block barrier needed)
-        uint8_t* lring = smem + L.region + align16(p.lay_chunk * 2);
-        constexpr int kSlot = LG::kBytes;               // bytes per token
-        constexpr int kStage = kNT * kSlot;
-        const int nst = (n_loc + kNT - 1) / kNT;
-        auto issue = [&](int j) {
-            const int i = j * kNT + tid;
-            if (j < nst && i < n_loc && i != app_i) {
-                uint8_t* dst = lring + (j % kLabStages) * kStage + tid * kSlot;
-                const uint8_t* src = lab + (size_t)(t0 + i) * kSlot;
-#pragma unroll
-                for (int o = 0; o < kSlot; o += 16) cp_async16(dst + o, src + o);
-            }
-        };
-#pragma unroll 1
-        for (int j = 0; j < kLabStages - 1; ++j) { issue(j); cp_async_commit(); }
+    if (use_ring) {
 #pragma unroll 1
         for (int j = 0; j < nst; ++j) {
             issue(j + kLabStages - 1);
@@ -455,7 +488,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
                 bits8[grp] = (uint8_t)flags;
                 for (uint32_t m = flags; m; m &= m - 1) {
                     const int i = grp * 8 + __ffs(m) - 1;
-                    const uint32_t low = score_key(rescore(i)) & 0xFFFFu;
+                    const uint32_t low = p.keep_low ? (uint32_t)low16[i] : score_key(rescore(i)) & 0xFFFFu;
                     keys[i] = (uint16_t)low;
                     atomicAdd(&histA[low >> 8], 1u);
                     const int slot = atomicAdd(&ctl[kCtlBL], 1);
@@ -523,8 +556,10 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         const int gpw = (((ngrp + kNW - 1) / kNW) + 31) & ~31;   // groups per warp
         const int wg0 = wid * gpw, wg1 = min(ngrp, wg0 + gpw);
         uint32_t ns = 0, nt = 0;
+        // each group's masks are kept (2 bytes) for the write pass below
         for (int grp = wg0 + lane; grp - lane < wg1; grp += 32) {
             const uint32_t m = grp < wg1 ? masks8(grp) : 0u;
+            if (grp < wg1) mcache[grp] = (uint16_t)m;
             ns += __popc(m & 255u);
             nt += __popc(m >> 8);
         }
@@ -569,7 +604,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         int cur_dst = -1;
         int* rl = nullptr;
         for (int grp = wg0 + lane; grp - lane < wg1; grp += 32) {
-            const uint32_t m = grp < wg1 ? masks8(grp) : 0u;
+            const uint32_t m = grp < wg1 ? (uint32_t)mcache[grp] : 0u;
             const uint32_t smk = m & 255u, tmk = m >> 8;
             const uint32_t pk = ((uint32_t)__popc(smk) << 16) | (uint32_t)__popc(tmk);
             const uint32_t incl = warp_incl_scan(pk);
@@ -605,6 +640,11 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     const int n_att = select_all ? n_loc : max(0, min(p.per, k_eff - rank * p.per));
     auto att_token = [&](int j) -> int { return select_all ? t0 + j : sel_list[j]; };
     float* wp_out = nullptr;  // this warp's partial (m, l, o) per head, [GT][D + 2]
+    auto write_out = [&](int h, int d, float res) {
+        const size_t oidx = (size_t)row * G * D + (size_t)h * D + d;
+        if (p.out_bf16) reinterpret_cast<uint16_t*>(p.out)[oidx] = f32_to_bf16_bits(res);
+        else reinterpret_cast<float*>(p.out)[oidx] = res;
+    };
     if constexpr (E::kBytes == 2) {
         // bf16 K/V: tensor cores (mma.sync, fp32 accumulate) on 8-token tiles.
         //   Z  = Q K^T   m16n8k16: rows = the group's heads (padded to 16),
@@ -842,6 +882,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     }
     }
     __syncthreads();
+    // merge the warps' states per head; a single-CTA row writes its output here
     for (int e = tid; e < G * D; e += kNT) {
         const int h = e / D, d = e - h * D;
         float M = -INFINITY;
@@ -859,14 +900,17 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
                 Lsum = fmaf(f, wp[D + 1], Lsum);
             }
         }
-        co[h * D + d] = O;
-        if (d == 0) { cm[h] = M; cl[h] = Lsum; }
+        if (N == 1) {
+            write_out(h, d, O / Lsum);
+        } else {
+            co[h * D + d] = O;
+            if (d == 0) { cm[h] = M; cl[h] = Lsum; }
+        }
     }
-    // [phase] 8
-    row_sync(cluster, N);                                            // CTA partials visible
-
-    // final merge across the cluster; CTA `rank` writes its slice of [G, D]
-    {
+    if (N > 1) {
+        // [phase] 8
+        row_sync(cluster, N);                                        // CTA partials visible
+        // final merge across the cluster; CTA `rank` writes its slice of [G, D]
         const int E_all = G * D;
         const int slice = (E_all + N - 1) / N;
         const int e0 = rank * slice, e1 = min(E_all, e0 + slice);
@@ -882,14 +926,11 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
                 O = fmaf(f, row_smem(cluster, N, co, r)[h * D + d], O);
                 Lsum = fmaf(f, row_smem(cluster, N, cl, r)[h], Lsum);
             }
-            const float res = O / Lsum;
-            const size_t oidx = (size_t)row * G * D + (size_t)h * D + d;
-            if (p.out_bf16) reinterpret_cast<uint16_t*>(p.out)[oidx] = f32_to_bf16_bits(res);
-            else reinterpret_cast<float*>(p.out)[oidx] = res;
+            write_out(h, d, O / Lsum);
         }
+        row_sync(cluster, N);                                        // keep smem alive for readers
     }
     // [phase] 9
-    row_sync(cluster, N);                                            // keep smem alive for readers
 }
 
 }  // namespace ds
