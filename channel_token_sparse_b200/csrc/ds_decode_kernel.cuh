@@ -77,7 +77,7 @@ __host__ __device__ inline int align16(int x) { return (x + 15) & ~15; }
 // (at most 8 * (128 + 2) floats) is later written into its own ring.
 constexpr int kAttStagesF32 = 4;
 // Label-streaming ring (fp labels): stages of one row per thread.
-constexpr int kLabStages = 6;
+constexpr int kLabStages = 8;
 __host__ __device__ constexpr int lab_ring_bytes(int label_row_bytes) { return kLabStages * 256 * label_row_bytes; }
 __host__ __device__ constexpr int att_stage_tokens(int row_bytes, int elem_bytes) {
     return elem_bytes == 2 ? 8 : (row_bytes >= 1024 ? 1 : 1024 / row_bytes);
@@ -118,7 +118,8 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int GT, int D, int C, i
 }
 
 // ctl[] slots
-enum { kCtlBin = 0, kCtlNeed = 1, kCtlCnt = 2, kCtlCS = 4, kCtlCT = 5, kCtlP = 6, kCtlTP = 7, kCtlBL = 8 };
+enum { kCtlBin = 0, kCtlNeed = 1, kCtlCnt = 2, kCtlCS = 4, kCtlCT = 5, kCtlP = 6, kCtlTP = 7, kCtlBL = 8,
+       kCtlTlo = 9, kCtlTie = 10 };
 
 // Row geometry of the label cache.
 template <typename TKV, int LK, int C>
@@ -309,7 +310,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         if (tid < C) idx_s[tid] = min(max(iv, 0), D - 1);
         histA[tid] = 0u;
         histB[tid] = 0u;
-        if (tid == 0) ctl[kCtlBL] = 0;
+        if (tid == 0) { ctl[kCtlBL] = 0; ctl[kCtlTie] = 0; }
     }
     __syncthreads();
     if (!p.dense) {
@@ -473,6 +474,9 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         T16 = (bA << 8) | ctl[kCtlBin];
         const int needB = ctl[kCtlNeed];
         refine = needB < ctl[kCtlCnt];
+        // a single-CTA row whose split bucket has at most kNT tokens ranks
+        // them exactly instead of running two more radix passes
+        const bool rank_mode = N == 1 && ctl[kCtlCnt] <= kNT;
         // [phase] 4
         if (refine) {
             // The k-th key's 16-bit bucket is split: re-score its tokens
@@ -490,11 +494,36 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
                     const int i = grp * 8 + __ffs(m) - 1;
                     const uint32_t low = p.keep_low ? (uint32_t)low16[i] : score_key(rescore(i)) & 0xFFFFu;
                     keys[i] = (uint16_t)low;
-                    atomicAdd(&histA[low >> 8], 1u);
+                    if (!rank_mode) atomicAdd(&histA[low >> 8], 1u);
                     const int slot = atomicAdd(&ctl[kCtlBL], 1);
                     if (slot < kBucketCap) blist[slot] = low | ((uint32_t)i << 16);
                 }
             }
+        }
+        if (refine && rank_mode) {
+            // rank of each bucket token by (low key bits desc, index asc); the
+            // needB-th gives the low threshold, and the tokens equal to it that
+            // rank inside are the ties to take
+            __syncthreads();
+            const int nbl = ctl[kCtlBL];
+            int my_low = -1, my_rank = 0;
+            if (tid < nbl) {
+                const uint32_t e = blist[tid];
+                my_low = (int)(e & 0xFFFFu);
+                const int my_idx = (int)(e >> 16);
+                for (int j = 0; j < nbl; ++j) {
+                    const uint32_t f = blist[j];
+                    const int lo = (int)(f & 0xFFFFu), ix = (int)(f >> 16);
+                    my_rank += (lo > my_low) || (lo == my_low && ix < my_idx);
+                }
+                if (my_rank == needB - 1) ctl[kCtlTlo] = my_low;
+            }
+            __syncthreads();
+            Tlo = ctl[kCtlTlo];
+            if (tid < nbl && my_low == Tlo && my_rank < needB) atomicAdd(&ctl[kCtlTie], 1);
+            __syncthreads();
+            r_tie = ctl[kCtlTie];
+        } else if (refine) {
             // [phase] 12
             row_sync(cluster, N);                                    // histograms C complete
             // [phase] 13

@@ -392,3 +392,31 @@ def test_decode_step_equals_append_then_decode(kv, label, d, c, hq, hkv, s, topk
     check_selection(sg.reshape(-1, topk), sel_ref.reshape(-1, topk), s_ref.reshape(-1, s), topk, s)
     o_ref = oracle.attention(di.q, di.k, di.v, kv, sg, hkv)
     assert np.abs(o1.cpu().numpy() - o_ref).max() <= OUT_ATOL
+
+
+@pytest.mark.parametrize("cluster,s,topk", [(1, 600, 100), (1, 3000, 700), (2, 3000, 700), (1, 2048, 1)])
+def test_exact_ties_small_buckets(cluster, s, topk):
+    """Integer label values make many exactly tied scores with small 16-bit
+    buckets (the in-bucket rank path for single-CTA rows, radix passes
+    otherwise); the selection must match the oracle's lowest-index rule."""
+    wl = synth.custom(b=1, hq=2, hkv=2, d=64, s=s, c=8, topk=topk, index=74)
+    di = synth.decode_inputs(wl)
+    r = np.random.default_rng(6)
+    di.k[:] = np.float32(r.integers(-8, 9, size=di.k.shape))
+    q = np.ones((1, 2, 64), np.float32)
+    idx = np.tile(np.arange(8, dtype=np.int32), (2, 1))
+    qd, kd, vd = to_dev(q, "f32"), to_dev(di.k, "f32"), to_dev(di.v, "f32")
+    idxd = torch.from_numpy(idx).cuda()
+    lab, _, _ = _gpu_label(kd, idxd, wl.s, wl)
+    ds.set_cluster(cluster)
+    try:
+        sel = torch.empty((1, 2, topk), dtype=torch.int32, device="cuda")
+        out = ds.sparse_decode(qd, kd, vd, lab, idxd, wl.s, topk, sel_out=sel)
+        torch.cuda.synchronize()
+    finally:
+        ds.set_cluster(0)
+    ref_lab = oracle.label_copy(di.k, "f32", idx, wl.s)
+    _, sel_ref, _ = oracle.sparse_decode(q, di.k, di.v, "f32", ref_lab, "f32", idx, wl.s, topk)
+    assert np.array_equal(sel.cpu().numpy(), sel_ref)
+    o_ref = oracle.attention(q, di.k, di.v, "f32", sel_ref, 2)
+    assert np.abs(out.cpu().numpy() - o_ref).max() <= OUT_ATOL
