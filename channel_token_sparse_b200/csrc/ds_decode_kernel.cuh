@@ -119,7 +119,7 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int GT, int D, int C, i
 
 // ctl[] slots
 enum { kCtlBin = 0, kCtlNeed = 1, kCtlCnt = 2, kCtlCS = 4, kCtlCT = 5, kCtlP = 6, kCtlTP = 7, kCtlBL = 8,
-       kCtlTlo = 9, kCtlTie = 10 };
+       kCtlTlo = 9, kCtlTie = 10, kCtlWarp = 16 /* kNW per-warp packed counts */ };
 
 // Row geometry of the label cache.
 template <typename TKV, int LK, int C>
@@ -477,18 +477,29 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         // a single-CTA row whose split bucket has at most kNT tokens ranks
         // them exactly instead of running two more radix passes
         const bool rank_mode = N == 1 && ctl[kCtlCnt] <= kNT;
+        // Warp w owns the contiguous key groups [wg0, wg1) for the refine
+        // sweep and the compaction; in each step lane l reads group
+        // wg0 + 32*step + l (conflict-free), so lane order is index order.
+        const int gpw = (((ngrp + kNW - 1) / kNW) + 31) & ~31;   // groups per warp
+        const int wg0 = wid * gpw, wg1 = min(ngrp, wg0 + gpw);
         // [phase] 4
         if (refine) {
-            // The k-th key's 16-bit bucket is split: re-score its tokens
-            // (bit-identical arithmetic), keep their low 16 key bits in place
-            // of the high ones, flag them, and list them for pass D.
-            for (int grp = tid; grp < ngrp; grp += kNT) {
+            // The k-th key's 16-bit bucket is split: take the low 16 key bits
+            // of its tokens (kept, or re-scored with bit-identical arithmetic)
+            // in place of the high ones, flag and list them; count each warp's
+            // keys above the bucket (selected outright) on the way.
+            uint32_t above_cnt = 0;
+            for (int grp = wg0 + lane; grp - lane < wg1; grp += 32) {
+                if (grp >= wg1) continue;
                 uint32_t w[4];
                 key8(grp, w);
                 uint32_t flags = 0;
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    if (grp * 8 + e < n_loc && kat(w, e) == T16) flags |= 1u << e;
+                for (int e = 0; e < 8; ++e) {
+                    const bool ok = grp * 8 + e < n_loc;
+                    if (ok && kat(w, e) == T16) flags |= 1u << e;
+                    above_cnt += ok && kat(w, e) > T16;
+                }
                 bits8[grp] = (uint8_t)flags;
                 for (uint32_t m = flags; m; m &= m - 1) {
                     const int i = grp * 8 + __ffs(m) - 1;
@@ -499,6 +510,8 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
                     if (slot < kBucketCap) blist[slot] = low | ((uint32_t)i << 16);
                 }
             }
+            above_cnt = __reduce_add_sync(0xffffffffu, above_cnt);
+            if (lane == 0) ctl[kCtlWarp + wid] = (int)(above_cnt << 16);
         }
         if (refine && rank_mode) {
             // rank of each bucket token by (low key bits desc, index asc); the
@@ -582,19 +595,34 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
             }
             return sm | (tm << 8);
         };
-        const int gpw = (((ngrp + kNW - 1) / kNW) + 31) & ~31;   // groups per warp
-        const int wg0 = wid * gpw, wg1 = min(ngrp, wg0 + gpw);
-        uint32_t ns = 0, nt = 0;
-        // each group's masks are kept (2 bytes) for the write pass below
-        for (int grp = wg0 + lane; grp - lane < wg1; grp += 32) {
-            const uint32_t m = grp < wg1 ? masks8(grp) : 0u;
-            if (grp < wg1) mcache[grp] = (uint16_t)m;
-            ns += __popc(m & 255u);
-            nt += __popc(m >> 8);
+        // Per-warp (selected, tie) counts. With a split bucket that is fully
+        // listed they follow from the refine sweep's counts plus the listed
+        // bucket tokens; otherwise a count pass classifies every key (and
+        // keeps each group's masks, 2 bytes, for the write pass).
+        const bool counts_known = refine && ctl[kCtlBL] <= kBucketCap;
+        if (counts_known) {
+            const int nbl = ctl[kCtlBL];
+            for (int j = tid; j < nbl; j += kNT) {
+                const uint32_t e = blist[j];
+                const int low = (int)(e & 0xFFFFu), i = (int)(e >> 16);
+                const int w = (i >> 3) / gpw;
+                if (low > Tlo) atomicAdd(&ctl[kCtlWarp + w], 1 << 16);
+                else if (low == Tlo) atomicAdd(&ctl[kCtlWarp + w], 1);
+            }
+            __syncthreads();
+            if (lane == 0) scan[wid] = (uint32_t)ctl[kCtlWarp + wid];
+        } else {
+            uint32_t ns = 0, nt = 0;
+            for (int grp = wg0 + lane; grp - lane < wg1; grp += 32) {
+                const uint32_t m = grp < wg1 ? masks8(grp) : 0u;
+                if (grp < wg1) mcache[grp] = (uint16_t)m;
+                ns += __popc(m & 255u);
+                nt += __popc(m >> 8);
+            }
+            ns = (uint32_t)__reduce_add_sync(0xffffffffu, ns);
+            nt = (uint32_t)__reduce_add_sync(0xffffffffu, nt);
+            if (lane == 0) scan[wid] = (ns << 16) | nt;
         }
-        ns = (uint32_t)__reduce_add_sync(0xffffffffu, ns);
-        nt = (uint32_t)__reduce_add_sync(0xffffffffu, nt);
-        if (lane == 0) scan[wid] = (ns << 16) | nt;
         __syncthreads();
         if (wid == 0) {
             const uint32_t x = lane < kNW ? scan[lane] : 0u;
@@ -633,7 +661,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         int cur_dst = -1;
         int* rl = nullptr;
         for (int grp = wg0 + lane; grp - lane < wg1; grp += 32) {
-            const uint32_t m = grp < wg1 ? (uint32_t)mcache[grp] : 0u;
+            const uint32_t m = grp < wg1 ? (counts_known ? masks8(grp) : (uint32_t)mcache[grp]) : 0u;
             const uint32_t smk = m & 255u, tmk = m >> 8;
             const uint32_t pk = ((uint32_t)__popc(smk) << 16) | (uint32_t)__popc(tmk);
             const uint32_t incl = warp_incl_scan(pk);
