@@ -43,13 +43,14 @@ def _load():
         _lib = C.CDLL(build())
         vp, i, d = C.c_void_p, C.c_int, C.c_double
         _lib.oracle_calibrate.argtypes = [vp, vp, i, i, i, i, i, i, i, i, vp, vp]
+        _lib.oracle_calibrate_criterion.argtypes = [vp, vp, i, i, i, i, i, i, i, i, i, i, vp, vp]
         _lib.oracle_label_copy.argtypes = [vp, i, vp, i, i, i, i, i, i, i, vp]
         _lib.oracle_label_int4.argtypes = [vp, i, vp, i, i, i, i, i, i, i, vp, vp, vp]
         _lib.oracle_label_int4_values.argtypes = [vp, vp, vp, i, i, i, i, vp]
         _lib.oracle_scores.argtypes = [vp, i, vp, vp, i, i, i, i, i, i, vp]
         _lib.oracle_topk.argtypes = [vp, i, i, i, vp]
         _lib.oracle_attention.argtypes = [vp, vp, vp, i, vp, i, i, i, i, i, i, d, vp]
-        for f in (_lib.oracle_calibrate, _lib.oracle_label_copy, _lib.oracle_label_int4,
+        for f in (_lib.oracle_calibrate, _lib.oracle_calibrate_criterion, _lib.oracle_label_copy, _lib.oracle_label_int4,
                   _lib.oracle_label_int4_values, _lib.oracle_scores, _lib.oracle_topk,
                   _lib.oracle_attention):
             f.restype = C.c_int
@@ -78,6 +79,24 @@ def calibrate(q_win: np.ndarray, k: np.ndarray, dtype: str, c: int):
     _check(_load().oracle_calibrate(_p(q_win), _p(k), _DT[dtype], n, hq, hkv, w, s, d, c,
                                     _p(ratio), _p(idx)), "calibrate")
     return ratio, idx
+
+
+CRITERIA = {"leank": 0, "q": 1, "k": 2, "qk": 3, "qk_chunked": 4}
+
+
+def calibrate_criterion(q_win: np.ndarray, k: np.ndarray, dtype: str, c: int, criterion: str,
+                        chunk: int = 0):
+    """Channel score [Hkv, D] under one outlier criterion and the heavy
+    channels idx [Hkv, C]; criterion in CRITERIA, chunk for "qk_chunked"."""
+    n, hq, w, d = q_win.shape
+    n2, hkv, s, d2 = k.shape
+    assert n == n2 and d == d2
+    score = np.zeros((hkv, d), dtype=np.float64)
+    idx = np.zeros((hkv, c), dtype=np.int32)
+    _check(_load().oracle_calibrate_criterion(_p(q_win), _p(k), _DT[dtype], n, hq, hkv, w, s, d, c,
+                                              CRITERIA[criterion], int(chunk), _p(score), _p(idx)),
+           "calibrate_criterion")
+    return score, idx
 
 
 def label_copy(k: np.ndarray, dtype: str, idx: np.ndarray, s: int, t_begin: int = 0,

@@ -11,7 +11,8 @@
  *           "离线校准" (offline calibration, label cache, 4-bit label cache) and
  *           "在线前向计算" (online decode: steps 1-3).
  *   [LeanK] "K通道静态性量化方法解析" (aitangshan.cn), §1.1 "通道重要性比率计算"
- *           (the channel importance ratio r_i).
+ *           (the channel importance ratio r_i) and §2.1 "与Double Sparsity的对比分析"
+ *           (Double Sparsity's chunked norm collection).
  *
  * Floating point is fp64 except the int4 quantiser, whose integer codes are a
  * decision taken in fp32 by the kernel; the oracle takes it in fp32 too.
@@ -139,6 +140,94 @@ int oracle_calibrate(const void* q_win, const void* k, int dtype,
 
     for (int g = 0; g < hkv; ++g) {
         for (int i = 0; i < d; ++i) { rk[i].r = ratio[(size_t)g * d + i]; rk[i].i = i; }
+        qsort(rk, (size_t)d, sizeof(ranked_t), cmp_ranked);
+        for (int j = 0; j < c; ++j) pick[j] = rk[j].i;
+        qsort(pick, (size_t)c, sizeof(int), cmp_int);
+        for (int j = 0; j < c; ++j) idx[(size_t)g * c + j] = pick[j];
+    }
+    free(Q); free(K); free(rk); free(pick);
+    return 0;
+}
+
+/* ------------------------------------- outlier criteria  ([DS] 离线校准;
+ *                                         [LeanK] §2.1 "与Double Sparsity的对比分析")
+ *
+ * [DS] lists channel strategies by outliers of the query, of the key and of
+ * query * key; [LeanK] §2.1 says DS collects norms of the QK product chunked
+ * along the context. Readings, for Q (the group's stacked windows, rows x d)
+ * and K (s x d) of one sample and kv head:
+ *   criterion 1 (Q-outlier):  score_i = L2 norm of the channel column Q[:, i]
+ *   criterion 2 (K-outlier):  score_i = L2 norm of K[:, i]
+ *   criterion 3 (QK-outlier): score_i = Frobenius norm of the channel's part
+ *                             of the product, Q[:, i] K[:, i]^T
+ *   criterion 4 (chunked):    the same norm taken over each context chunk
+ *                             [j*chunk, min(s, (j+1)*chunk)) and summed over j
+ *   criterion 0:              the LeanK ratio of oracle_calibrate.
+ * Each is averaged over the samples and ranked like oracle_calibrate. The
+ * norms are written out entrywise as defined (no closed form).
+ */
+int oracle_calibrate_criterion(const void* q_win, const void* k, int dtype,
+                               int n, int hq, int hkv, int w, int s, int d, int c,
+                               int criterion, int chunk,
+                               double* score /* [hkv, d] */, int32_t* idx /* [hkv, c] */) {
+    if (criterion == 0)
+        return oracle_calibrate(q_win, k, dtype, n, hq, hkv, w, s, d, c, score, idx);
+    if (criterion < 0 || criterion > 4 || (criterion == 4 && chunk < 1)) return 1;
+    if (n < 1 || hkv < 1 || hq % hkv || w < 1 || s < 1 || d < 1 || c < 1 || c > d)
+        return 1;
+    const int G = hq / hkv;
+    const int rows = G * w;
+    double* Q = (double*)malloc(sizeof(double) * (size_t)rows * d);
+    double* K = (double*)malloc(sizeof(double) * (size_t)s * d);
+    ranked_t* rk = (ranked_t*)malloc(sizeof(ranked_t) * (size_t)d);
+    int* pick = (int*)malloc(sizeof(int) * (size_t)c);
+    if (!Q || !K || !rk || !pick) { free(Q); free(K); free(rk); free(pick); return 2; }
+
+    for (int g = 0; g < hkv; ++g)
+        for (int i = 0; i < d; ++i) score[(size_t)g * d + i] = 0.0;
+
+    for (int ns = 0; ns < n; ++ns) {
+        for (int g = 0; g < hkv; ++g) {
+            for (int j = 0; j < G; ++j)
+                for (int t = 0; t < w; ++t)
+                    for (int i = 0; i < d; ++i) {
+                        size_t src = (((size_t)ns * hq + (size_t)g * G + j) * w + t) * d + i;
+                        Q[((size_t)j * w + t) * d + i] = elem(q_win, dtype, src);
+                    }
+            for (int t = 0; t < s; ++t)
+                for (int i = 0; i < d; ++i)
+                    K[(size_t)t * d + i] = elem(k, dtype, (((size_t)ns * hkv + g) * s + t) * d + i);
+
+            for (int i = 0; i < d; ++i) {
+                double v = 0.0;
+                if (criterion == 1) {
+                    double a = 0.0;
+                    for (int row = 0; row < rows; ++row) a += Q[(size_t)row * d + i] * Q[(size_t)row * d + i];
+                    v = sqrt(a);
+                } else if (criterion == 2) {
+                    double a = 0.0;
+                    for (int t = 0; t < s; ++t) a += K[(size_t)t * d + i] * K[(size_t)t * d + i];
+                    v = sqrt(a);
+                } else {
+                    const int len = criterion == 3 ? s : chunk;
+                    for (int t0 = 0; t0 < s; t0 += len) {
+                        const int t1 = t0 + len < s ? t0 + len : s;
+                        double a = 0.0;
+                        for (int row = 0; row < rows; ++row)
+                            for (int t = t0; t < t1; ++t) {
+                                double e = Q[(size_t)row * d + i] * K[(size_t)t * d + i];
+                                a += e * e;
+                            }
+                        v += sqrt(a);
+                    }
+                }
+                score[(size_t)g * d + i] += v / (double)n;
+            }
+        }
+    }
+
+    for (int g = 0; g < hkv; ++g) {
+        for (int i = 0; i < d; ++i) { rk[i].r = score[(size_t)g * d + i]; rk[i].i = i; }
         qsort(rk, (size_t)d, sizeof(ranked_t), cmp_ranked);
         for (int j = 0; j < c; ++j) pick[j] = rk[j].i;
         qsort(pick, (size_t)c, sizeof(int), cmp_int);

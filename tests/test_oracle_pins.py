@@ -314,3 +314,107 @@ def test_int4_scores_equal_dequantised_dot():
         ze.view(np.float16).astype(np.float64)[..., :, None]
     qsum = di.q[0].astype(np.float64).sum(0)[idx[0]]
     np.testing.assert_allclose(s[0, 0], deq[0, 0] @ qsum, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------- calibration criteria
+
+_CRIT = ("q", "k", "qk", "qk_chunked")
+
+
+def test_criteria_hand_cases():
+    for case in _gold("calib_criteria_hand.json")["cases"]:
+        q = np.array(case["q"], np.float32)[None, None]
+        k = np.array(case["k"], np.float32)[None, None]
+        for name, key in (("q", "q_outlier"), ("k", "k_outlier"), ("qk", "qk_outlier"),
+                          ("qk_chunked", "qk_chunked"), ("leank", "leank")):
+            if key not in case:
+                continue
+            score, idx = oracle.calibrate_criterion(q, k, "f32", case["c"], name, case["chunk"])
+            np.testing.assert_allclose(score[0], case[key]["score"], rtol=1e-14)
+            assert idx[0].tolist() == case[key]["idx"], name
+
+
+def _stack_group(q_win, g, G):
+    """[N, Hq, W, D] -> per sample the group's windows stacked, [N, G*W, D]."""
+    n, hq, w, d = q_win.shape
+    return q_win[:, g * G:(g + 1) * G].reshape(n, G * w, d).astype(np.float64)
+
+
+def test_criteria_match_library_norms():
+    """Column norms and outer-product norms from numpy, averaged over samples,
+    with a GQA group of two query heads per kv head."""
+    r = np.random.default_rng(21)
+    n, hq, hkv, w, s, d = 3, 4, 2, 5, 37, 16
+    q = r.standard_normal((n, hq, w, d)).astype(np.float32)
+    k = r.standard_normal((n, hkv, s, d)).astype(np.float32)
+    G = hq // hkv
+    for g in range(hkv):
+        Qs, Ks = _stack_group(q, g, G), k[:, g].astype(np.float64)
+        want = {
+            "q": np.mean([np.linalg.norm(Qs[j], axis=0) for j in range(n)], axis=0),
+            "k": np.mean([np.linalg.norm(Ks[j], axis=0) for j in range(n)], axis=0),
+            "qk": np.mean([[np.linalg.norm(np.outer(Qs[j][:, i], Ks[j][:, i]), "fro") for i in range(d)]
+                           for j in range(n)], axis=0),
+            "qk_chunked": np.mean([[sum(np.linalg.norm(np.outer(Qs[j][:, i], Ks[j][t0:t0 + 10, i]), "fro")
+                                        for t0 in range(0, s, 10)) for i in range(d)]
+                                   for j in range(n)], axis=0),
+        }
+        for name in _CRIT:
+            score, idx = oracle.calibrate_criterion(q, k, "f32", 5, name, 10)
+            np.testing.assert_allclose(score[g], want[name], rtol=1e-12)
+            top = sorted(np.lexsort((np.arange(d), -want[name]))[:5].tolist())
+            assert idx[g].tolist() == top, name
+
+
+def test_chunked_criterion_limits():
+    """One chunk spanning the context equals the QK-outlier score; chunks of
+    one token give ||Q[:,i]|| * sum_t |K[t,i]| (closed form)."""
+    r = np.random.default_rng(22)
+    q = r.standard_normal((2, 1, 4, 8)).astype(np.float32)
+    k = r.standard_normal((2, 1, 13, 8)).astype(np.float32)
+    a, _ = oracle.calibrate_criterion(q, k, "f32", 3, "qk")
+    b, _ = oracle.calibrate_criterion(q, k, "f32", 3, "qk_chunked", 13)
+    c, _ = oracle.calibrate_criterion(q, k, "f32", 3, "qk_chunked", 1000)
+    np.testing.assert_allclose(a, b, rtol=1e-14)
+    np.testing.assert_allclose(a, c, rtol=1e-14)
+    one, _ = oracle.calibrate_criterion(q, k, "f32", 3, "qk_chunked", 1)
+    Q, K = q[:, 0].astype(np.float64), k[:, 0].astype(np.float64)
+    closed = np.mean(np.linalg.norm(Q, axis=1) * np.abs(K).sum(axis=1), axis=0)
+    np.testing.assert_allclose(one[0], closed, rtol=1e-12)
+
+
+def test_leank_criterion_and_single_sample_qk_ranking():
+    """Criterion "leank" is the LeanK ratio; with one sample the ratio is the
+    QK-outlier score over a per-head constant, so both rank alike."""
+    r = np.random.default_rng(23)
+    q = r.standard_normal((1, 2, 6, 16)).astype(np.float32)
+    k = r.standard_normal((1, 1, 20, 16)).astype(np.float32)
+    ra, ia = oracle.calibrate(q, k, "f32", 6)
+    rb, ib = oracle.calibrate_criterion(q, k, "f32", 6, "leank")
+    np.testing.assert_array_equal(ra, rb)
+    assert ia.tolist() == ib.tolist()
+    sq, iq = oracle.calibrate_criterion(q, k, "f32", 6, "qk")
+    Qs, K = q[0].reshape(12, 16).astype(np.float64), k[0, 0].astype(np.float64)
+    np.testing.assert_allclose(sq[0], ra[0] * np.linalg.norm(Qs @ K.T, "fro"), rtol=1e-12)
+    assert iq.tolist() == ia.tolist()
+
+
+def test_criteria_separate_query_and_key_outliers():
+    """Outliers planted only in K are found by the K criterion and missed by
+    the Q criterion, and the other way round (catches swapped operands)."""
+    r = np.random.default_rng(24)
+    q = r.standard_normal((2, 2, 8, 32)).astype(np.float32)
+    k = r.standard_normal((2, 1, 64, 32)).astype(np.float32)
+    kch, qch = [3, 9, 17, 30], [1, 12, 20, 25]
+    k[..., kch] *= 8
+    q[..., qch] *= 8
+    _, ik = oracle.calibrate_criterion(q, k, "f32", 4, "k")
+    _, iq = oracle.calibrate_criterion(q, k, "f32", 4, "q")
+    assert ik[0].tolist() == kch and iq[0].tolist() == qch
+
+
+def test_criteria_reject_bad_arguments():
+    q = np.ones((1, 1, 2, 4), np.float32)
+    k = np.ones((1, 1, 3, 4), np.float32)
+    with pytest.raises(Exception):
+        oracle.calibrate_criterion(q, k, "f32", 2, "qk_chunked", 0)
