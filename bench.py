@@ -327,10 +327,11 @@ def run_ours(args, wl, rank, local_rank, world):
 
     # dense baseline on the same cache: our dense kernel and torch SDPA
     dense_ms, sdpa_ms = dense_baselines(wl, q, k, v, out, flush, stream)
+    offload = offload_timing(wl, q, k, v, idx, lab, sc, ze, out, flush, stream) if args.offload else None
 
     res = dict(step_ms=step_ms, total_s=total_s, max_s=max_s,
                wall_s=wall1 - wall0, e2e_s=e2e_max, h2d=h2d, d2h=d2h, prefill_ms=prefill_ms,
-               clocks=sampler.summary(), dense_ms=dense_ms, sdpa_ms=sdpa_ms,
+               clocks=sampler.summary(), dense_ms=dense_ms, sdpa_ms=sdpa_ms, offload=offload,
                plan=ds.plan(wl.b, wl.hq, wl.hkv, wl.s, wl.d, wl.c, wl.topk,
                             ds.DS_BF16 if wl.kv_dtype == "bf16" else ds.DS_F32,
                             ds.DS_INT4 if wl.label_dtype == "int4" else
@@ -390,6 +391,38 @@ def dense_baselines(wl, q, k, v, out, flush, stream, reps=20):
     except Exception:  # noqa: BLE001
         pass
     return dense_ms, sdpa_ms
+
+
+def offload_timing(wl, q, k, v, idx, lab, sc, ze, out, flush, stream, reps=20):
+    """Double Sparsity's offloading mode: the same decode step with the K/V
+    caches in pinned host memory (label cache, query and output on the GPU),
+    the selected rows crossing the host link; and dense decode over the same
+    host caches (every row crosses). Medians of `reps` launches (ms)."""
+    import torch
+
+    import channel_token_sparse_b200 as ds
+
+    kh, vh = k.cpu().pin_memory(), v.cpu().pin_memory()
+
+    def timed(fn):
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                fn()
+            ts = []
+            for _ in range(reps):
+                flush()
+                a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                fn()
+                b_.record()
+                ts.append((a, b_))
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b_) for a, b_ in ts)
+
+    sparse_ms = timed(lambda: ds.decode_step(q, kh, vh, lab, idx, wl.s, wl.topk, lscale=sc, lzero=ze, out=out))
+    dense_ms = timed(lambda: ds.dense_decode(q, kh, vh, wl.s, out=out))
+    del kh, vh
+    return sparse_ms, dense_ms
 
 
 def barrier():
@@ -490,6 +523,8 @@ def main():
     ap.add_argument("--config", type=int, default=1, help="workload index (0-4)")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=8, help="rows per reference-arm step")
+    ap.add_argument("--offload", action="store_true",
+                    help="also time the step with the K/V caches in pinned host memory")
     ap.add_argument("--flush", default="copy", choices=["copy", "fill"],
                     help="L2 eviction between timed steps: D2D copy or fill kernel")
     args = ap.parse_args()
@@ -568,6 +603,15 @@ def report(args, wl, r, world):
                                 "gbs": prefill_bytes(wl) / (r["prefill_ms"] / 1e3) / 1e9},
         "wall_s_timed_region": r["wall_s"],
     }
+    if r["offload"]:
+        sp_ms, dn_ms = r["offload"]
+        esz = 2 if wl.kv_dtype == "bf16" else 4
+        link = wl.b * wl.hkv * (2 * min(wl.topk, wl.s) + 1) * wl.d * esz
+        line["offload"] = {"kv_in": "pinned host memory", "sparse_step_us": sp_ms * 1e3,
+                           "tokens_per_s": wl.b / (sp_ms / 1e3), "host_link_bytes": link,
+                           "host_link_gbs": link / (sp_ms / 1e3) / 1e9,
+                           "dense_us": dn_ms * 1e3, "dense_host_link_bytes": 2 * wl.b * wl.hkv * wl.s * wl.d * esz,
+                           "speedup_vs_dense": dn_ms / sp_ms}
     return line
 
 

@@ -23,6 +23,7 @@ LIB_PATH = os.path.join(HERE, "libds.so")
 
 DS_OK, DS_ERR_INVALID_ARG, DS_ERR_UNSUPPORTED, DS_ERR_CUDA, DS_ERR_WORKSPACE = range(5)
 DS_F32, DS_BF16, DS_F16, DS_INT4 = range(4)
+DS_CRIT_LEANK_RATIO, DS_CRIT_Q_OUTLIER, DS_CRIT_K_OUTLIER, DS_CRIT_QK_OUTLIER, DS_CRIT_QK_CHUNKED = range(5)
 
 # every C-ABI entry point: name -> (restype, argtypes)
 _vp, _i, _f, _sz = C.c_void_p, C.c_int, C.c_float, C.c_size_t
@@ -32,12 +33,16 @@ SIGNATURES = {
     "ds_calibrate_workspace_size": (_i, [_i, _i, _i, _i, _i, _i, C.POINTER(_sz)]),
     "ds_calibrate_channels": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp]),
     "ds_calibrate_channels_noalloc": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "ds_calibrate_channels_criterion": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp,
+                                             _vp, _sz, _vp]),
     "ds_build_label_cache": (_i, [_vp, _i, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _vp]),
     "ds_append_label": (_i, [_vp, _i, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _vp]),
     "ds_sparse_decode": (_i, [_vp, _vp, _vp, _i, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
                               _f, _vp, _i, _vp, _vp, _vp]),
     "ds_decode_step": (_i, [_vp, _vp, _vp, _i, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
                             _f, _vp, _i, _vp, _vp, _vp]),
+    "ds_decode_step_varlen": (_i, [_vp, _vp, _vp, _i, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                   _i, _f, _vp, _i, _vp, _vp, _vp]),
     "ds_sparse_decode_plan": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, _i, C.POINTER(_i), C.POINTER(_i),
                                    C.POINTER(_i)]),
     "ds_sparse_decode_set_cluster": (None, [_i]),
@@ -95,6 +100,29 @@ def _torch():
 
 def _ptr(t):
     return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _ptr_kv(t):
+    """Device address of a key/value cache: a CUDA tensor, or a pinned host
+    tensor mapped into the device's address space (DS-Offload: the kernels
+    then read the rows they need over the host link)."""
+    if t.is_cuda:
+        return C.c_void_p(t.data_ptr())
+    if not t.is_pinned():
+        raise ValueError("a key/value cache in host memory must be pinned")
+    from cuda.bindings import runtime as rt
+    err, dptr = rt.cudaHostGetDevicePointer(t.data_ptr(), 0)
+    if err != rt.cudaError_t.cudaSuccess:
+        raise ValueError(f"pinned host cache is not mapped for the device: {err}")
+    return C.c_void_p(int(dptr))
+
+
+def _need_cuda_or_pinned(*ts):
+    for t in ts:
+        if not (t.is_cuda or t.is_pinned()):
+            raise ValueError("key/value caches must be CUDA tensors or pinned host tensors")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
 
 
 def _stream(stream=None):
@@ -161,6 +189,26 @@ def calibrate_channels(q_win, k, c: int, ratio_out=None, idx_out=None, ws=None, 
     return idx_out, ratio_out
 
 
+def calibrate_channels_criterion(q_win, k, c: int, criterion: int, chunk: int = 0, score_out=None,
+                                 idx_out=None, ws=None, stream=None):
+    """Heavy channels ranked by one of the DS_CRIT_* criteria. Returns (idx, score)."""
+    torch = _torch()
+    _need_cuda(q_win, k)
+    n, hq, w, d = q_win.shape
+    _, hkv, s, _ = k.shape
+    if idx_out is None:
+        idx_out = torch.empty((hkv, c), dtype=torch.int32, device=k.device)
+    if score_out is None:
+        score_out = torch.empty((hkv, d), dtype=torch.float32, device=k.device)
+    nbytes = calibrate_workspace_size(n, hq, hkv, w, s, d)
+    if ws is None:
+        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=k.device)
+    _check(lib().ds_calibrate_channels_criterion(_ptr(q_win), _ptr(k), _kv_dtype(k), n, hq, hkv, w, s, d,
+                                                 c, int(criterion), int(chunk), _ptr(score_out),
+                                                 _ptr(idx_out), _ptr(ws), ws.numel(), _stream(stream)))
+    return idx_out, score_out
+
+
 def calibrate_channels_noalloc(q_win, k, c: int, ratio_out, idx_out, stream=None):
     """ds_calibrate_channels with the library's fixed scratch instead of a
     workspace (for callers that cannot allocate device memory); the outputs
@@ -183,23 +231,26 @@ def _label_args(label, lscale, lzero, kdt):
 
 
 def build_label_cache(k, idx, s: int, label, lscale=None, lzero=None, stream=None):
-    """Fill label rows [0, s) from the key cache k [B, Hkv, S_cap, D]."""
-    _need_cuda(k, idx, label, lscale, lzero)
+    """Fill label rows [0, s) from the key cache k [B, Hkv, S_cap, D] (device,
+    or pinned host memory)."""
+    _need_cuda_or_pinned(k)
+    _need_cuda(idx, label, lscale, lzero)
     b, hkv, s_cap, d = k.shape
     c = idx.shape[1]
     kdt = _kv_dtype(k)
-    _check(lib().ds_build_label_cache(_ptr(k), kdt, _ptr(idx), b, hkv, s, s_cap, d, c, _ptr(label),
+    _check(lib().ds_build_label_cache(_ptr_kv(k), kdt, _ptr(idx), b, hkv, s, s_cap, d, c, _ptr(label),
                                       _label_args(label, lscale, lzero, kdt), _ptr(lscale),
                                       _ptr(lzero), _stream(stream)))
 
 
 def append_label(k, idx, pos: int, label, lscale=None, lzero=None, stream=None):
     """Fill label row `pos` from k[:, :, pos]."""
-    _need_cuda(k, idx, label, lscale, lzero)
+    _need_cuda_or_pinned(k)
+    _need_cuda(idx, label, lscale, lzero)
     b, hkv, s_cap, d = k.shape
     c = idx.shape[1]
     kdt = _kv_dtype(k)
-    _check(lib().ds_append_label(_ptr(k), kdt, _ptr(idx), b, hkv, pos, s_cap, d, c, _ptr(label),
+    _check(lib().ds_append_label(_ptr_kv(k), kdt, _ptr(idx), b, hkv, pos, s_cap, d, c, _ptr(label),
                                  _label_args(label, lscale, lzero, kdt), _ptr(lscale), _ptr(lzero),
                                  _stream(stream)))
 
@@ -219,7 +270,8 @@ def sparse_decode(q, k, v, label, idx, s: int, topk: int, lscale=None, lzero=Non
                   out_dtype=None, sm_scale: float = 0.0, sel_out=None, score_out=None, stream=None):
     """One Double Sparsity decode step; returns out [B, Hq, D]."""
     torch = _torch()
-    _need_cuda(q, k, v, label, idx, lscale, lzero, out, sel_out, score_out)
+    _need_cuda_or_pinned(k, v)
+    _need_cuda(q, label, idx, lscale, lzero, out, sel_out, score_out)
     b, hq, d = q.shape
     _, hkv, s_cap, _ = k.shape
     c = idx.shape[1]
@@ -227,7 +279,7 @@ def sparse_decode(q, k, v, label, idx, s: int, topk: int, lscale=None, lzero=Non
     if out is None:
         out = torch.empty((b, hq, d), dtype=out_dtype or torch.float32, device=q.device)
     odt = DS_F32 if out.dtype == torch.float32 else DS_BF16
-    _check(lib().ds_sparse_decode(_ptr(q), _ptr(k), _ptr(v), kdt, _ptr(label),
+    _check(lib().ds_sparse_decode(_ptr(q), _ptr_kv(k), _ptr_kv(v), kdt, _ptr(label),
                                   _label_args(label, lscale, lzero, kdt), _ptr(lscale), _ptr(lzero),
                                   _ptr(idx), b, hq, hkv, s, s_cap, d, c, topk, float(sm_scale),
                                   _ptr(out), odt, _ptr(sel_out), _ptr(score_out), _stream(stream)))
@@ -239,7 +291,8 @@ def decode_step(q, k, v, label, idx, s: int, topk: int, lscale=None, lzero=None,
     """append_label(pos = s - 1) followed by sparse_decode, in one launch;
     returns out [B, Hq, D]."""
     torch = _torch()
-    _need_cuda(q, k, v, label, idx, lscale, lzero, out, sel_out, score_out)
+    _need_cuda_or_pinned(k, v)
+    _need_cuda(q, label, idx, lscale, lzero, out, sel_out, score_out)
     b, hq, d = q.shape
     _, hkv, s_cap, _ = k.shape
     c = idx.shape[1]
@@ -247,22 +300,45 @@ def decode_step(q, k, v, label, idx, s: int, topk: int, lscale=None, lzero=None,
     if out is None:
         out = torch.empty((b, hq, d), dtype=out_dtype or torch.float32, device=q.device)
     odt = DS_F32 if out.dtype == torch.float32 else DS_BF16
-    _check(lib().ds_decode_step(_ptr(q), _ptr(k), _ptr(v), kdt, _ptr(label),
+    _check(lib().ds_decode_step(_ptr(q), _ptr_kv(k), _ptr_kv(v), kdt, _ptr(label),
                                 _label_args(label, lscale, lzero, kdt), _ptr(lscale), _ptr(lzero),
                                 _ptr(idx), b, hq, hkv, s, s_cap, d, c, topk, float(sm_scale),
                                 _ptr(out), odt, _ptr(sel_out), _ptr(score_out), _stream(stream)))
     return out
 
 
+def decode_step_varlen(q, k, v, label, idx, seq_lens, s_max: int, topk: int, lscale=None, lzero=None, out=None,
+                       out_dtype=None, sm_scale: float = 0.0, sel_out=None, score_out=None, stream=None):
+    """decode_step with a per-batch-entry token count seq_lens [B] (int32,
+    device); returns out [B, Hq, D]."""
+    torch = _torch()
+    _need_cuda_or_pinned(k, v)
+    _need_cuda(q, label, idx, seq_lens, lscale, lzero, out, sel_out, score_out)
+    b, hq, d = q.shape
+    _, hkv, s_cap, _ = k.shape
+    c = idx.shape[1]
+    kdt = _kv_dtype(k)
+    if out is None:
+        out = torch.empty((b, hq, d), dtype=out_dtype or torch.float32, device=q.device)
+    odt = DS_F32 if out.dtype == torch.float32 else DS_BF16
+    _check(lib().ds_decode_step_varlen(_ptr(q), _ptr_kv(k), _ptr_kv(v), kdt, _ptr(label),
+                                       _label_args(label, lscale, lzero, kdt), _ptr(lscale), _ptr(lzero),
+                                       _ptr(idx), _ptr(seq_lens), b, hq, hkv, s_max, s_cap, d, c, topk,
+                                       float(sm_scale), _ptr(out), odt, _ptr(sel_out), _ptr(score_out),
+                                       _stream(stream)))
+    return out
+
+
 def dense_decode(q, k, v, s: int, out=None, out_dtype=None, sm_scale: float = 0.0, stream=None):
     """Dense decode attention over tokens [0, s) (measurement baseline)."""
     torch = _torch()
-    _need_cuda(q, k, v, out)
+    _need_cuda_or_pinned(k, v)
+    _need_cuda(q, out)
     b, hq, d = q.shape
     _, hkv, s_cap, _ = k.shape
     if out is None:
         out = torch.empty((b, hq, d), dtype=out_dtype or torch.float32, device=q.device)
     odt = DS_F32 if out.dtype == torch.float32 else DS_BF16
-    _check(lib().ds_dense_decode(_ptr(q), _ptr(k), _ptr(v), _kv_dtype(k), b, hq, hkv, s, s_cap, d,
+    _check(lib().ds_dense_decode(_ptr(q), _ptr_kv(k), _ptr_kv(v), _kv_dtype(k), b, hq, hkv, s, s_cap, d,
                                  float(sm_scale), _ptr(out), odt, _stream(stream)))
     return out

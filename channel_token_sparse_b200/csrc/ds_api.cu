@@ -260,6 +260,34 @@ ds_status ds_calibrate_channels(const void* q_win, const void* k, ds_dtype dt, i
     return DS_OK;
 }
 
+ds_status ds_calibrate_channels_criterion(const void* q_win, const void* k, ds_dtype dt, int n_samples,
+                                          int hq, int hkv, int w, int s, int d, int c,
+                                          ds_calib_criterion criterion, int chunk, float* score_out,
+                                          int32_t* idx_out, void* ws, size_t ws_bytes,
+                                          cudaStream_t stream) {
+    size_t need = 0;
+    ds_status r = ds_calibrate_workspace_size(n_samples, hq, hkv, w, s, d, &need);
+    if (r != DS_OK) return r;
+    if (!kv_dtype_ok(dt)) return fail(DS_ERR_UNSUPPORTED, "dtype %d (supported: f32, bf16)", (int)dt);
+    if (c < 1 || c > d) return fail(DS_ERR_INVALID_ARG, "need 1 <= c (%d) <= d (%d)", c, d);
+    if ((int)criterion < DS_CRIT_LEANK_RATIO || (int)criterion > DS_CRIT_QK_CHUNKED)
+        return fail(DS_ERR_INVALID_ARG, "unknown criterion %d", (int)criterion);
+    if (criterion == DS_CRIT_QK_CHUNKED && chunk < 1)
+        return fail(DS_ERR_INVALID_ARG, "chunk (%d) must be >= 1", chunk);
+    if (hq / hkv * (long long)w > (1 << 20)) return fail(DS_ERR_UNSUPPORTED, "window too large");
+    if (!q_win || !k || !idx_out || !ws) return fail(DS_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(q_win) || !aligned16(k) || !aligned16(idx_out) || !aligned16(ws) ||
+        (score_out && !aligned16(score_out)))
+        return fail(DS_ERR_INVALID_ARG, "pointer not 16-byte aligned");
+    if (ws_bytes < need) return fail(DS_ERR_WORKSPACE, "workspace %zu B < required %zu B", ws_bytes, need);
+    ds::CalibArgs a{q_win, k, dt == DS_BF16, n_samples, hq, hkv, w, s, d, c, score_out, idx_out, ws};
+    a.criterion = (int)criterion;
+    a.chunk = criterion == DS_CRIT_QK_CHUNKED ? chunk : 0;
+    cudaError_t e = ds::launch_calib(a, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "calibration launch");
+    return DS_OK;
+}
+
 ds_status ds_calibrate_channels_noalloc(const void* q_win, const void* k, ds_dtype dt, int n_samples,
                                         int hq, int hkv, int w, int s, int d, int c, float* ratio_out,
                                         int32_t* idx_out, cudaStream_t stream) {
@@ -323,7 +351,7 @@ ds_status sparse_decode_impl(const void* q, const void* k, const void* v, ds_dty
                              ds_dtype label_dt, const uint16_t* lscale, const uint16_t* lzero,
                              const int32_t* idx, int b, int hq, int hkv, int s, int s_cap, int d, int c,
                              int topk, float sm_scale, void* out, ds_dtype out_dt, int32_t* sel_out,
-                             float* score_out, bool append, cudaStream_t stream) {
+                             float* score_out, bool append, const int32_t* seq_lens, cudaStream_t stream) {
     ds_status r = check_common(b, hq, hkv, s, s_cap, d, kvdt);
     if (r != DS_OK) return r;
     if ((r = check_label(kvdt, label_dt, c, d, label, lscale, lzero)) != DS_OK) return r;
@@ -345,7 +373,9 @@ ds_status sparse_decode_impl(const void* q, const void* k, const void* v, ds_dty
     ds::DecodeKernel kern = pick_kernel(kvdt, label_dt == DS_INT4, d, c, GT);
     if (!kern) return fail(DS_ERR_UNSUPPORTED, "no kernel for d=%d c=%d G=%d", d, c, G);
     ds::DecodeParams p{};
+    if (seq_lens && !aligned16(seq_lens)) return fail(DS_ERR_INVALID_ARG, "seq_lens not 16-byte aligned");
     p.q = q; p.k = k; p.v = v; p.label = label; p.lscale = lscale; p.lzero = lzero; p.idx = idx;
+    p.seq_lens = seq_lens;
     p.out = out; p.sel_out = sel_out; p.score_out = score_out;
     p.hkv = hkv; p.G = G; p.s = s; p.s_cap = s_cap; p.topk = topk;
     p.chunk = pl.chunk; p.lay_chunk = pl.lay_chunk; p.per = pl.per;
@@ -370,7 +400,7 @@ ds_status ds_sparse_decode(const void* q, const void* k, const void* v, ds_dtype
                            int s_cap, int d, int c, int topk, float sm_scale, void* out,
                            ds_dtype out_dt, int32_t* sel_out, float* score_out, cudaStream_t stream) {
     return sparse_decode_impl(q, k, v, kvdt, label, label_dt, lscale, lzero, idx, b, hq, hkv, s, s_cap, d, c,
-                              topk, sm_scale, out, out_dt, sel_out, score_out, false, stream);
+                              topk, sm_scale, out, out_dt, sel_out, score_out, false, nullptr, stream);
 }
 
 ds_status ds_decode_step(const void* q, const void* k, const void* v, ds_dtype kvdt, void* label,
@@ -379,7 +409,17 @@ ds_status ds_decode_step(const void* q, const void* k, const void* v, ds_dtype k
                          void* out, ds_dtype out_dt, int32_t* sel_out, float* score_out,
                          cudaStream_t stream) {
     return sparse_decode_impl(q, k, v, kvdt, label, label_dt, lscale, lzero, idx, b, hq, hkv, s, s_cap, d, c,
-                              topk, sm_scale, out, out_dt, sel_out, score_out, true, stream);
+                              topk, sm_scale, out, out_dt, sel_out, score_out, true, nullptr, stream);
+}
+
+ds_status ds_decode_step_varlen(const void* q, const void* k, const void* v, ds_dtype kvdt, void* label,
+                                ds_dtype label_dt, uint16_t* lscale, uint16_t* lzero, const int32_t* idx,
+                                const int32_t* seq_lens, int b, int hq, int hkv, int s_max, int s_cap, int d,
+                                int c, int topk, float sm_scale, void* out, ds_dtype out_dt, int32_t* sel_out,
+                                float* score_out, cudaStream_t stream) {
+    if (!seq_lens) return fail(DS_ERR_INVALID_ARG, "seq_lens is NULL");
+    return sparse_decode_impl(q, k, v, kvdt, label, label_dt, lscale, lzero, idx, b, hq, hkv, s_max, s_cap, d, c,
+                              topk, sm_scale, out, out_dt, sel_out, score_out, true, seq_lens, stream);
 }
 
 ds_status ds_dense_decode(const void* q, const void* k, const void* v, ds_dtype kvdt, int b, int hq,

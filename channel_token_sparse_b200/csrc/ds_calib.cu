@@ -11,6 +11,13 @@
 // entries of Q K^T (fp32 dot products, fp64 accumulation) into the caller's
 // workspace, then one CTA per kv head forms r (mean over samples) and ranks
 // the channels (ties to the lower channel index).
+//
+// The same sums also rank channels by the outlier criteria that "大模型稀疏化
+// 技术原理：Double Sparsity" lists beside its offline calibration (Q-, K- and
+// QK-outlier), and by the chunked-norm collection "K通道静态性量化方法解析"
+// §2.1 attributes to Double Sparsity: the per-channel score is the column
+// norm ||Q[:,i]||, ||K[:,i]||, the product of both, or ||Q[:,i]|| times the sum
+// over context chunks of ||K[chunk, i]||.
 #include <mutex>
 
 #include "ds_common.cuh"
@@ -30,6 +37,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kCalNT) ds_calib_partial_kernel(const T* __restrict__ qwin,
                                                                    const T* __restrict__ k, int hq,
                                                                    int hkv, int w, int s,
+                                                                   bool k_sums, bool den_sums,
                                                                    double* __restrict__ ws) {
     using E = Elem<T>;
     __shared__ float ks[kCalTile][D + 1];
@@ -49,7 +57,7 @@ __global__ void __launch_bounds__(kCalNT) ds_calib_partial_kernel(const T* __res
     }
     __syncthreads();
     // per-channel sum of squares of this key tile
-    for (int i = threadIdx.x; i < D; i += kCalNT) {
+    for (int i = threadIdx.x; k_sums && i < D; i += kCalNT) {
         double a = 0.0;
         for (int t = 0; t < nt; ++t) a += (double)ks[t][i] * (double)ks[t][i];
         atomicAdd(&blk[D + i], a);
@@ -78,7 +86,7 @@ __global__ void __launch_bounds__(kCalNT) ds_calib_partial_kernel(const T* __res
                 atomicAdd(&blk[i], a);
             }
         }
-        for (int e = threadIdx.x; e < kCalTile * kCalTile; e += kCalNT) {
+        for (int e = threadIdx.x; den_sums && e < kCalTile * kCalTile; e += kCalNT) {
             const int rr = e / kCalTile, t = e - rr * kCalTile;
             if (rr < nr && t < nt) {
                 float dot = 0.f;
@@ -98,9 +106,40 @@ __global__ void __launch_bounds__(kCalNT) ds_calib_partial_kernel(const T* __res
     }
 }
 
+// Sum over the context chunks [t0, t0 + chunk) of ||K[chunk, i]|| per channel,
+// into the k slot of the workspace (chunked-norm criterion). One CTA per
+// (chunk, kv head, sample); each of the kCalNT / D token lanes sums a strided
+// part of the chunk, and the lanes are added in a fixed order.
+template <typename T, int D>
+__global__ void __launch_bounds__(kCalNT) ds_calib_kchunk_kernel(const T* __restrict__ k, int hkv,
+                                                                  int s, int chunk,
+                                                                  double* __restrict__ ws) {
+    using E = Elem<T>;
+    constexpr int L = kCalNT / D;
+    __shared__ double part[L][D];
+    const int n = blockIdx.z, g = blockIdx.y;
+    const int t0 = blockIdx.x * chunk;
+    const int t1 = min(s, t0 + chunk);
+    const int i = threadIdx.x % D, l = threadIdx.x / D;
+    const T* kb = k + ((size_t)n * hkv + g) * (size_t)s * D;
+    double a = 0.0;
+    for (int t = t0 + l; t < t1; t += L) {
+        const double x = (double)E::to_f32(kb[(size_t)t * D + i]);
+        a += x * x;
+    }
+    part[l][i] = a;
+    __syncthreads();
+    if (l == 0) {
+        double sq = 0.0;
+        for (int j = 0; j < L; ++j) sq += part[j][i];
+        atomicAdd(&ws[((size_t)n * hkv + g) * (2 * D + 1) + D + i], sqrt(sq));
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(D) ds_calib_rank_kernel(const double* __restrict__ ws, int n,
-                                                          int hkv, int c, float* __restrict__ ratio,
+                                                          int hkv, int c, int criterion,
+                                                          float* __restrict__ ratio,
                                                           int32_t* __restrict__ idx) {
     __shared__ double r[D];
     __shared__ uint32_t scan[D / 32 + 1];
@@ -108,8 +147,17 @@ __global__ void __launch_bounds__(D) ds_calib_rank_kernel(const double* __restri
     double acc = 0.0;
     for (int ns = 0; ns < n; ++ns) {
         const double* blk = ws + ((size_t)ns * hkv + g) * (2 * D + 1);
-        const double den = sqrt(blk[2 * D]);
-        const double v = den > 0.0 ? sqrt(blk[i]) * sqrt(blk[D + i]) / den : 0.0;
+        double v;
+        switch (criterion) {
+        case kCritQ: v = sqrt(blk[i]); break;
+        case kCritK: v = sqrt(blk[D + i]); break;
+        case kCritQK: v = sqrt(blk[i]) * sqrt(blk[D + i]); break;
+        case kCritQKChunked: v = sqrt(blk[i]) * blk[D + i]; break;
+        default: {
+            const double den = sqrt(blk[2 * D]);
+            v = den > 0.0 ? sqrt(blk[i]) * sqrt(blk[D + i]) / den : 0.0;
+        }
+        }
         acc += v / (double)n;
     }
     r[i] = acc;
@@ -129,13 +177,21 @@ template <typename T, int D>
 static cudaError_t launch_calib_t(const CalibArgs& a, cudaStream_t st) {
     cudaError_t e = cudaMemsetAsync(a.ws, 0, calib_workspace_bytes(a.n, a.hkv, D), st);
     if (e != cudaSuccess) return e;
+    const bool chunked = a.criterion == kCritQKChunked;
     dim3 grid((a.s + kCalTile - 1) / kCalTile, a.hkv, a.n);
     ds_calib_partial_kernel<T, D><<<grid, kCalNT, 0, st>>>(
         reinterpret_cast<const T*>(a.q_win), reinterpret_cast<const T*>(a.k), a.hq, a.hkv, a.w, a.s,
-        reinterpret_cast<double*>(a.ws));
+        !chunked, a.criterion == kCritLeanK, reinterpret_cast<double*>(a.ws));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (chunked) {
+        dim3 cg((a.s + a.chunk - 1) / a.chunk, a.hkv, a.n);
+        ds_calib_kchunk_kernel<T, D><<<cg, kCalNT, 0, st>>>(reinterpret_cast<const T*>(a.k), a.hkv,
+                                                             a.s, a.chunk,
+                                                             reinterpret_cast<double*>(a.ws));
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     ds_calib_rank_kernel<D><<<a.hkv, D, 0, st>>>(reinterpret_cast<const double*>(a.ws), a.n, a.hkv,
-                                                  a.c, a.ratio, a.idx);
+                                                  a.c, a.criterion, a.ratio, a.idx);
     return cudaGetLastError();
 }
 

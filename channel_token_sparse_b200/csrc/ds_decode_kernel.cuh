@@ -46,10 +46,11 @@ struct DecodeParams {
     const uint16_t* lscale;
     const uint16_t* lzero;
     const int32_t* idx;
+    const int32_t* seq_lens;  // [b] tokens per batch entry, or null (all rows have s)
     void* out;
     int32_t* sel_out;
     float* score_out;
-    int hkv, G, s, s_cap, topk;
+    int hkv, G, s, s_cap, topk;  // s: tokens per row (the maximum when seq_lens is given)
     int chunk;     // tokens per CTA, multiple of 32
     int lay_chunk; // chunk used to size shared memory (0 in dense mode)
     int per;       // selected tokens attended per CTA (ceil(min(topk,s) / N))
@@ -238,7 +239,9 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     int* sel_list = reinterpret_cast<int*>(smem + L.sel);
     uint16_t* keys = reinterpret_cast<uint16_t*>(smem + L.region);
 
-    const int s = p.s;
+    // tokens of this row: one length for all rows, or per batch entry
+    // (clamped into [1, s]) when the caller gives seq_lens
+    const int s = p.seq_lens ? min(max(p.seq_lens[row / p.hkv], 1), p.s) : p.s;
     const int t0 = rank * p.chunk;
     const int n_loc = max(0, min(s, t0 + p.chunk) - t0);
     const size_t row_tok = (size_t)row * (size_t)p.s_cap;  // first token of this row in the caches
@@ -401,7 +404,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
             if (p.keep_low) low16[i] = (uint16_t)key;
             atomicAdd(&histA[key >> 24], 1u);
         }
-        if (p.score_out) p.score_out[(size_t)row * s + t0 + i] = sv;
+        if (p.score_out) p.score_out[(size_t)row * p.s + t0 + i] = sv;
     };
     if (use_ring) {
 #pragma unroll 1

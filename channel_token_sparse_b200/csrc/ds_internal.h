@@ -28,6 +28,9 @@ struct LabelArgs {
 };
 cudaError_t launch_label(const LabelArgs& a, cudaStream_t st);
 
+// Channel ranking criteria (values of ds_calib_criterion).
+enum { kCritLeanK = 0, kCritQ = 1, kCritK = 2, kCritQK = 3, kCritQKChunked = 4 };
+
 struct CalibArgs {
     const void* q_win;
     const void* k;
@@ -36,6 +39,8 @@ struct CalibArgs {
     float* ratio;
     int32_t* idx;
     void* ws;
+    int criterion = kCritLeanK;
+    int chunk = 0;  // context chunk length (kCritQKChunked only)
 };
 size_t calib_workspace_bytes(int n, int hkv, int d);
 cudaError_t launch_calib(const CalibArgs& a, cudaStream_t st);

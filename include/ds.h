@@ -98,6 +98,40 @@ DS_API ds_status ds_calibrate_channels(const void* q_win, const void* k, ds_dtyp
                                 float* ratio_out, int32_t* idx_out,
                                 void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* Channel ranking criteria for ds_calibrate_channels_criterion. The
+ * Double Sparsity page ("大模型稀疏化技术原理：Double Sparsity", 离线校准)
+ * lists outlier strategies by query, key and query*key; "K通道静态性量化方法
+ * 解析" §2.1 says Double Sparsity's offline collection takes norms of the QK
+ * product chunked along the context. Per sample n and kv head g (Q_g, K_g as
+ * for ds_calibrate_channels), channel i scores
+ *   DS_CRIT_LEANK_RATIO  ||Q_g[:,i] K_g[:,i]^T||_F / ||Q_g K_g^T||_F  (= ds_calibrate_channels)
+ *   DS_CRIT_Q_OUTLIER    ||Q_g[:,i]||_2
+ *   DS_CRIT_K_OUTLIER    ||K_g[:,i]||_2
+ *   DS_CRIT_QK_OUTLIER   ||Q_g[:,i] K_g[:,i]^T||_F  (= ||Q_g[:,i]|| ||K_g[:,i]||)
+ *   DS_CRIT_QK_CHUNKED   sum over chunks [j*chunk, min(s, (j+1)*chunk)) of
+ *                        ||Q_g[:,i] K_g[chunk,i]^T||_F
+ * and the score is the mean over samples. The activation-outlier strategy
+ * ranks channels of the layer input, before the projections, and is not
+ * offered: this library starts from Q and K. */
+typedef enum {
+    DS_CRIT_LEANK_RATIO = 0,
+    DS_CRIT_Q_OUTLIER = 1,
+    DS_CRIT_K_OUTLIER = 2,
+    DS_CRIT_QK_OUTLIER = 3,
+    DS_CRIT_QK_CHUNKED = 4
+} ds_calib_criterion;
+
+/* ds_calibrate_channels with a choice of criterion. `chunk` (>= 1) is the
+ * context chunk length of DS_CRIT_QK_CHUNKED and is ignored otherwise.
+ * score_out [hkv, d] float32 (or NULL) receives the mean score; idx_out and
+ * the workspace are as for ds_calibrate_channels (same size). Ties go to the
+ * lower channel. DS_ERR_INVALID_ARG for an unknown criterion or chunk < 1. */
+DS_API ds_status ds_calibrate_channels_criterion(const void* q_win, const void* k, ds_dtype dt,
+                                                 int n_samples, int hq, int hkv, int w, int s,
+                                                 int d, int c, ds_calib_criterion criterion,
+                                                 int chunk, float* score_out, int32_t* idx_out,
+                                                 void* ws, size_t ws_bytes, cudaStream_t stream);
+
 /* Calibration for callers that cannot allocate device memory -- code that
  * runs while a CUDA graph is being captured, plugins whose host framework owns
  * every allocation, or runtimes with a fixed device budget. It has no
@@ -179,6 +213,22 @@ DS_API ds_status ds_decode_step(const void* q, const void* k, const void* v, ds_
                                 int b, int hq, int hkv, int s, int s_cap, int d, int c, int topk,
                                 float sm_scale, void* out, ds_dtype out_dt,
                                 int32_t* sel_out, float* score_out, cudaStream_t stream);
+
+/* ds_decode_step for a batch of sequences of different lengths (serving):
+ * seq_lens [b] (device, int32) gives each batch entry's token count s_b, and
+ * kernels clamp it into [1, s_max]. Row (b, g) appends its token s_b - 1 and
+ * attends over its own top-min(topk, s_b) of tokens [0, s_b); s_b <= topk is
+ * dense attention over the row, the fallback of the pages' SGLang threshold
+ * rule. score_out is laid out [b, hkv, s_max] with entries t >= s_b
+ * untouched, and sel_out entries past min(topk, s_b) are -1. The launch is
+ * planned for s_max. */
+DS_API ds_status ds_decode_step_varlen(const void* q, const void* k, const void* v, ds_dtype kvdt,
+                                       void* label, ds_dtype label_dt,
+                                       uint16_t* lscale, uint16_t* lzero, const int32_t* idx,
+                                       const int32_t* seq_lens,
+                                       int b, int hq, int hkv, int s_max, int s_cap, int d, int c,
+                                       int topk, float sm_scale, void* out, ds_dtype out_dt,
+                                       int32_t* sel_out, float* score_out, cudaStream_t stream);
 
 /* Launch plan of ds_sparse_decode for a shape (host only, launches nothing):
  * CTAs per thread-block cluster (one cluster per (b, kv head)), tokens per
