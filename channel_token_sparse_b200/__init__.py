@@ -23,6 +23,7 @@ LIB_PATH = os.path.join(HERE, "libds.so")
 
 DS_OK, DS_ERR_INVALID_ARG, DS_ERR_UNSUPPORTED, DS_ERR_CUDA, DS_ERR_WORKSPACE = range(5)
 DS_F32, DS_BF16, DS_F16, DS_INT4 = range(4)
+DS_FALLBACK_PER_ENTRY, DS_FALLBACK_BATCH = range(2)
 DS_CRIT_LEANK_RATIO, DS_CRIT_Q_OUTLIER, DS_CRIT_K_OUTLIER, DS_CRIT_QK_OUTLIER, DS_CRIT_QK_CHUNKED = range(5)
 
 # every C-ABI entry point: name -> (restype, argtypes)
@@ -42,7 +43,7 @@ SIGNATURES = {
     "ds_decode_step": (_i, [_vp, _vp, _vp, _i, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
                             _f, _vp, _i, _vp, _vp, _vp]),
     "ds_decode_step_varlen": (_i, [_vp, _vp, _vp, _i, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
-                                   _i, _f, _vp, _i, _vp, _vp, _vp]),
+                                   _i, _i, _i, _f, _vp, _i, _vp, _vp, _vp]),
     "ds_sparse_decode_plan": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, _i, C.POINTER(_i), C.POINTER(_i),
                                    C.POINTER(_i)]),
     "ds_sparse_decode_set_cluster": (None, [_i]),
@@ -308,9 +309,10 @@ def decode_step(q, k, v, label, idx, s: int, topk: int, lscale=None, lzero=None,
 
 
 def decode_step_varlen(q, k, v, label, idx, seq_lens, s_max: int, topk: int, lscale=None, lzero=None, out=None,
-                       out_dtype=None, sm_scale: float = 0.0, sel_out=None, score_out=None, stream=None):
+                       out_dtype=None, sm_scale: float = 0.0, sel_out=None, score_out=None,
+                       sparse_threshold: int = 0, fallback: int = DS_FALLBACK_PER_ENTRY, stream=None):
     """decode_step with a per-batch-entry token count seq_lens [B] (int32,
-    device); returns out [B, Hq, D]."""
+    device) and the short-entry fallback rule; returns out [B, Hq, D]."""
     torch = _torch()
     _need_cuda_or_pinned(k, v)
     _need_cuda(q, label, idx, seq_lens, lscale, lzero, out, sel_out, score_out)
@@ -323,7 +325,8 @@ def decode_step_varlen(q, k, v, label, idx, seq_lens, s_max: int, topk: int, lsc
     odt = DS_F32 if out.dtype == torch.float32 else DS_BF16
     _check(lib().ds_decode_step_varlen(_ptr(q), _ptr_kv(k), _ptr_kv(v), kdt, _ptr(label),
                                        _label_args(label, lscale, lzero, kdt), _ptr(lscale), _ptr(lzero),
-                                       _ptr(idx), _ptr(seq_lens), b, hq, hkv, s_max, s_cap, d, c, topk,
+                                       _ptr(idx), _ptr(seq_lens), int(sparse_threshold), int(fallback),
+                                       b, hq, hkv, s_max, s_cap, d, c, topk,
                                        float(sm_scale), _ptr(out), odt, _ptr(sel_out), _ptr(score_out),
                                        _stream(stream)))
     return out

@@ -351,7 +351,8 @@ ds_status sparse_decode_impl(const void* q, const void* k, const void* v, ds_dty
                              ds_dtype label_dt, const uint16_t* lscale, const uint16_t* lzero,
                              const int32_t* idx, int b, int hq, int hkv, int s, int s_cap, int d, int c,
                              int topk, float sm_scale, void* out, ds_dtype out_dt, int32_t* sel_out,
-                             float* score_out, bool append, const int32_t* seq_lens, cudaStream_t stream) {
+                             float* score_out, bool append, const int32_t* seq_lens, int threshold,
+                             int batch_rule, cudaStream_t stream) {
     ds_status r = check_common(b, hq, hkv, s, s_cap, d, kvdt);
     if (r != DS_OK) return r;
     if ((r = check_label(kvdt, label_dt, c, d, label, lscale, lzero)) != DS_OK) return r;
@@ -376,6 +377,9 @@ ds_status sparse_decode_impl(const void* q, const void* k, const void* v, ds_dty
     if (seq_lens && !aligned16(seq_lens)) return fail(DS_ERR_INVALID_ARG, "seq_lens not 16-byte aligned");
     p.q = q; p.k = k; p.v = v; p.label = label; p.lscale = lscale; p.lzero = lzero; p.idx = idx;
     p.seq_lens = seq_lens;
+    p.nb = b;
+    p.threshold = threshold;
+    p.batch_rule = batch_rule;
     p.out = out; p.sel_out = sel_out; p.score_out = score_out;
     p.hkv = hkv; p.G = G; p.s = s; p.s_cap = s_cap; p.topk = topk;
     p.chunk = pl.chunk; p.lay_chunk = pl.lay_chunk; p.per = pl.per;
@@ -400,7 +404,7 @@ ds_status ds_sparse_decode(const void* q, const void* k, const void* v, ds_dtype
                            int s_cap, int d, int c, int topk, float sm_scale, void* out,
                            ds_dtype out_dt, int32_t* sel_out, float* score_out, cudaStream_t stream) {
     return sparse_decode_impl(q, k, v, kvdt, label, label_dt, lscale, lzero, idx, b, hq, hkv, s, s_cap, d, c,
-                              topk, sm_scale, out, out_dt, sel_out, score_out, false, nullptr, stream);
+                              topk, sm_scale, out, out_dt, sel_out, score_out, false, nullptr, 0, 0, stream);
 }
 
 ds_status ds_decode_step(const void* q, const void* k, const void* v, ds_dtype kvdt, void* label,
@@ -409,17 +413,22 @@ ds_status ds_decode_step(const void* q, const void* k, const void* v, ds_dtype k
                          void* out, ds_dtype out_dt, int32_t* sel_out, float* score_out,
                          cudaStream_t stream) {
     return sparse_decode_impl(q, k, v, kvdt, label, label_dt, lscale, lzero, idx, b, hq, hkv, s, s_cap, d, c,
-                              topk, sm_scale, out, out_dt, sel_out, score_out, true, nullptr, stream);
+                              topk, sm_scale, out, out_dt, sel_out, score_out, true, nullptr, 0, 0, stream);
 }
 
 ds_status ds_decode_step_varlen(const void* q, const void* k, const void* v, ds_dtype kvdt, void* label,
                                 ds_dtype label_dt, uint16_t* lscale, uint16_t* lzero, const int32_t* idx,
-                                const int32_t* seq_lens, int b, int hq, int hkv, int s_max, int s_cap, int d,
-                                int c, int topk, float sm_scale, void* out, ds_dtype out_dt, int32_t* sel_out,
-                                float* score_out, cudaStream_t stream) {
+                                const int32_t* seq_lens, int sparse_threshold, ds_fallback fallback, int b,
+                                int hq, int hkv, int s_max, int s_cap, int d, int c, int topk, float sm_scale,
+                                void* out, ds_dtype out_dt, int32_t* sel_out, float* score_out,
+                                cudaStream_t stream) {
     if (!seq_lens) return fail(DS_ERR_INVALID_ARG, "seq_lens is NULL");
+    if (sparse_threshold < 0) return fail(DS_ERR_INVALID_ARG, "sparse_threshold (%d) < 0", sparse_threshold);
+    if (fallback != DS_FALLBACK_PER_ENTRY && fallback != DS_FALLBACK_BATCH)
+        return fail(DS_ERR_INVALID_ARG, "unknown fallback rule %d", (int)fallback);
     return sparse_decode_impl(q, k, v, kvdt, label, label_dt, lscale, lzero, idx, b, hq, hkv, s_max, s_cap, d, c,
-                              topk, sm_scale, out, out_dt, sel_out, score_out, true, seq_lens, stream);
+                              topk, sm_scale, out, out_dt, sel_out, score_out, true, seq_lens, sparse_threshold,
+                              fallback == DS_FALLBACK_BATCH ? 1 : 0, stream);
 }
 
 ds_status ds_dense_decode(const void* q, const void* k, const void* v, ds_dtype kvdt, int b, int hq,

@@ -46,7 +46,7 @@ struct DecodeParams {
     const uint16_t* lscale;
     const uint16_t* lzero;
     const int32_t* idx;
-    const int32_t* seq_lens;  // [b] tokens per batch entry, or null (all rows have s)
+    const int32_t* seq_lens;  // [nb] tokens per batch entry, or null (all rows have s)
     void* out;
     int32_t* sel_out;
     float* score_out;
@@ -61,6 +61,11 @@ struct DecodeParams {
     float qscale;  // sm_scale * log2(e)
     int out_bf16;
     int dense;     // 1: attend every token, no label / scores / selection
+    // with seq_lens: entries shorter than `threshold` attend all their tokens;
+    // batch_rule = 1 applies the rule to the whole batch instead (every entry
+    // attends all its tokens when the longest is shorter than `threshold` or
+    // the shortest is shorter than topk)
+    int nb, threshold, batch_rule;
 };
 
 // Shared-memory carve-up (bytes), identical on host and device.
@@ -247,7 +252,22 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     const size_t row_tok = (size_t)row * (size_t)p.s_cap;  // first token of this row in the caches
     const TKV* qrow = reinterpret_cast<const TKV*>(p.q) + (size_t)row * G * D;
     const int k_eff = min(p.topk, s);
-    const bool select_all = p.dense || p.topk >= s;
+    bool select_all = p.dense || p.topk >= s;
+    if (p.seq_lens) {  // the fallback rule for short entries
+        if (p.batch_rule) {
+            int any_short = 0, any_long = 0;
+            for (int j = threadIdx.x; j < p.nb; j += kNT) {
+                const int len = min(max(p.seq_lens[j], 1), p.s);
+                any_short |= len < p.topk;
+                any_long |= len >= p.threshold;
+            }
+            any_short = __syncthreads_or(any_short);
+            any_long = __syncthreads_or(any_long);
+            select_all = select_all || any_short || !any_long;
+        } else {
+            select_all = select_all || s < p.threshold;
+        }
+    }
 
     // [phase] 0
     const uint8_t* lab = reinterpret_cast<const uint8_t*>(p.label) + row_tok * LG::kBytes;
@@ -690,9 +710,14 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         // [phase] 20
         row_sync(cluster, N);                                        // selection lists complete
     } else if (p.sel_out) {
-        for (int i = tid; i < n_loc; i += kNT) p.sel_out[(size_t)row * p.topk + t0 + i] = t0 + i;
-        if (rank == 0)
-            for (int j = s + tid; j < p.topk; j += kNT) p.sel_out[(size_t)row * p.topk + j] = -1;
+        // every token is attended: listed when they fit, else the row is all -1
+        if (s <= p.topk) {
+            for (int i = tid; i < n_loc; i += kNT) p.sel_out[(size_t)row * p.topk + t0 + i] = t0 + i;
+            if (rank == 0)
+                for (int j = s + tid; j < p.topk; j += kNT) p.sel_out[(size_t)row * p.topk + j] = -1;
+        } else if (rank == 0) {
+            for (int j = tid; j < p.topk; j += kNT) p.sel_out[(size_t)row * p.topk + j] = -1;
+        }
     }
 
     // [phase] 6

@@ -214,18 +214,33 @@ DS_API ds_status ds_decode_step(const void* q, const void* k, const void* v, ds_
                                 float sm_scale, void* out, ds_dtype out_dt,
                                 int32_t* sel_out, float* score_out, cudaStream_t stream);
 
+/* When a batch entry is decoded with every one of its tokens instead of its
+ * top-k (the pages' SGLang section: --ds-sparse-decode-threshold and the
+ * heavy-token count decide when Double Sparsity is not used).
+ *   DS_FALLBACK_PER_ENTRY  entry b attends all its tokens when
+ *                          s_b <= topk or s_b < sparse_threshold; the other
+ *                          entries of the batch still select topk tokens.
+ *   DS_FALLBACK_BATCH      the rule as SGLang states it, for the whole batch:
+ *                          every entry attends all its tokens when
+ *                          max_b s_b < sparse_threshold or min_b s_b < topk. */
+typedef enum { DS_FALLBACK_PER_ENTRY = 0, DS_FALLBACK_BATCH = 1 } ds_fallback;
+
 /* ds_decode_step for a batch of sequences of different lengths (serving):
  * seq_lens [b] (device, int32) gives each batch entry's token count s_b, and
  * kernels clamp it into [1, s_max]. Row (b, g) appends its token s_b - 1 and
- * attends over its own top-min(topk, s_b) of tokens [0, s_b); s_b <= topk is
- * dense attention over the row, the fallback of the pages' SGLang threshold
- * rule. score_out is laid out [b, hkv, s_max] with entries t >= s_b
- * untouched, and sel_out entries past min(topk, s_b) are -1. The launch is
- * planned for s_max. */
+ * attends over its own top-min(topk, s_b) of tokens [0, s_b), or over all of
+ * [0, s_b) when the fallback rule says so (sparse_threshold >= 0; 0 disables
+ * the threshold part). score_out is laid out [b, hkv, s_max] with entries
+ * t >= s_b untouched. sel_out: the selected tokens, ascending, padded with
+ * -1; a row that attends all its tokens lists them when s_b <= topk and is
+ * all -1 otherwise. The launch is planned for s_max.
+ * DS_ERR_INVALID_ARG for seq_lens == NULL, a negative threshold or an
+ * unknown rule. */
 DS_API ds_status ds_decode_step_varlen(const void* q, const void* k, const void* v, ds_dtype kvdt,
                                        void* label, ds_dtype label_dt,
                                        uint16_t* lscale, uint16_t* lzero, const int32_t* idx,
-                                       const int32_t* seq_lens,
+                                       const int32_t* seq_lens, int sparse_threshold,
+                                       ds_fallback fallback,
                                        int b, int hq, int hkv, int s_max, int s_cap, int d, int c,
                                        int topk, float sm_scale, void* out, ds_dtype out_dt,
                                        int32_t* sel_out, float* score_out, cudaStream_t stream);

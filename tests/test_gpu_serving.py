@@ -2,7 +2,8 @@
 
 - per-batch-entry sequence lengths (ds_decode_step_varlen), each row checked
   against the oracle run on that entry alone with its own length, including
-  rows short enough that every token is attended;
+  rows short enough that every token is attended, and the threshold rule for
+  short entries (per entry, or for the whole batch as SGLang states it);
 - key/value caches in pinned host memory read by the kernels over the host
   link (Double Sparsity's offloading mode), bit-identical to device caches;
 - the channel criteria of ds_calibrate_channels_criterion (Q-, K-, QK-outlier,
@@ -119,6 +120,58 @@ def test_varlen_rows_match_oracle_per_entry(kv, label, d, c, hq, hkv, s_max, top
         assert err <= OUT_ATOL, f"entry {bb}: output max-abs error {err}"
 
 
+def _expected_all_tokens(seq_lens, topk, threshold, rule):
+    """Which entries attend every token (the SGLang threshold rule of the
+    Double Sparsity page, per entry or for the whole batch)."""
+    if rule == ds.DS_FALLBACK_BATCH:
+        whole = max(seq_lens) < threshold or min(seq_lens) < topk
+        return [whole or sb <= topk for sb in seq_lens]
+    return [sb <= topk or sb < threshold for sb in seq_lens]
+
+
+@pytest.mark.parametrize("seq_lens,threshold,rule", [
+    ([3000, 1700, 900, 100], 1000, ds.DS_FALLBACK_PER_ENTRY),
+    ([3000, 1700, 900, 200], 0, ds.DS_FALLBACK_BATCH),      # shortest < topk: the batch goes dense
+    ([3000, 1700, 900, 300], 3500, ds.DS_FALLBACK_BATCH),   # longest < threshold: dense
+    ([3000, 1700, 900, 300], 2000, ds.DS_FALLBACK_BATCH),   # neither: every entry sparse
+])
+def test_fallback_rule(seq_lens, threshold, rule):
+    kv, label, d, c, hq, hkv, s_max, topk = "bf16", "bf16", 128, 16, 8, 4, 3000, 256
+    b = len(seq_lens)
+    wl = synth.custom(b=b, hq=hq, hkv=hkv, d=d, s=s_max, c=c, topk=topk, kv_dtype=kv, label_dtype=label,
+                      n_outlier=16, outlier_scale=6.0, index=84)
+    di = synth.decode_inputs(wl, s_cap=s_max + 8)
+    idx = _idx_random(wl, 12)
+    qd, kd, vd = (to_dev(x, kv) for x in (di.q, di.k, di.v))
+    idxd = torch.from_numpy(idx).cuda()
+    lab, sc, ze = _label_alloc(kd, wl)
+    for bb, sb in enumerate(seq_lens):
+        ds.build_label_cache(kd[bb:bb + 1], idxd, sb - 1, lab[bb:bb + 1])
+    lens = torch.tensor(seq_lens, dtype=torch.int32, device="cuda")
+    sel = torch.full((b, hkv, topk), -7, dtype=torch.int32, device="cuda")
+    out = ds.decode_step_varlen(qd, kd, vd, lab, idxd, lens, s_max, topk, sel_out=sel,
+                                sparse_threshold=threshold, fallback=rule)
+    torch.cuda.synchronize()
+    out_h, sel_h = out.cpu().numpy(), sel.cpu().numpy()
+    for bb, (sb, dense) in enumerate(zip(seq_lens, _expected_all_tokens(seq_lens, topk, threshold, rule))):
+        kb, vb, qb = (np.ascontiguousarray(x[bb:bb + 1]) for x in (di.k, di.v, di.q))
+        ref_label = oracle.build_label(kb, kv, label, idx, sb)
+        if dense:
+            every = np.broadcast_to(np.arange(sb, dtype=np.int32), (1, hkv, sb)).copy()
+            o_ref = oracle.attention(qb, kb, vb, kv, every, hkv)
+            want = np.full((hkv, topk), -1, np.int32)
+            if sb <= topk:
+                want[:, :sb] = np.arange(sb)
+            assert np.array_equal(sel_h[bb], want), f"entry {bb}: sel_out of an all-token row"
+        else:
+            _, sel_ref, s_ref = oracle.sparse_decode(qb, kb, vb, kv, ref_label, label, idx, sb, topk)
+            check_selection(sel_h[bb].reshape(-1, topk), sel_ref.reshape(-1, topk), s_ref.reshape(-1, sb),
+                            topk, sb)
+            o_ref = oracle.attention(qb, kb, vb, kv, sel_h[bb:bb + 1], hkv)
+        err = np.abs(out_h[bb:bb + 1] - o_ref).max()
+        assert err <= OUT_ATOL, f"entry {bb} (all tokens: {dense}): output max-abs error {err}"
+
+
 def test_varlen_uniform_lengths_equal_decode_step():
     """All entries at s_max: bit-identical to ds_decode_step."""
     wl = synth.custom(b=3, hq=8, hkv=4, d=128, s=4000, c=16, topk=256, kv_dtype="bf16",
@@ -145,11 +198,16 @@ def test_varlen_rejects_missing_lengths():
     lab = torch.zeros((1, 2, 64, 8), device="cuda")
     idx = torch.zeros((2, 8), dtype=torch.int32, device="cuda")
     out = torch.zeros((1, 2, 64), device="cuda")
-    st = ds.lib().ds_decode_step_varlen(q.data_ptr(), k.data_ptr(), k.data_ptr(), ds.DS_F32, lab.data_ptr(),
-                                        ds.DS_F32, None, None, idx.data_ptr(), None, 1, 2, 2, 64, 64,
-                                        64, 8, 16, 0.0, out.data_ptr(), ds.DS_F32, None, None,
-                                        torch.cuda.current_stream().cuda_stream)
-    assert st == ds.DS_ERR_INVALID_ARG
+    lens = torch.full((1,), 64, dtype=torch.int32, device="cuda")
+
+    def call(seq_lens, threshold=0, rule=ds.DS_FALLBACK_PER_ENTRY):
+        return ds.lib().ds_decode_step_varlen(q.data_ptr(), k.data_ptr(), k.data_ptr(), ds.DS_F32, lab.data_ptr(),
+                                              ds.DS_F32, None, None, idx.data_ptr(), seq_lens, threshold, rule,
+                                              1, 2, 2, 64, 64, 64, 8, 16, 0.0, out.data_ptr(), ds.DS_F32, None,
+                                              None, torch.cuda.current_stream().cuda_stream)
+    assert call(None) == ds.DS_ERR_INVALID_ARG
+    assert call(lens.data_ptr(), threshold=-1) == ds.DS_ERR_INVALID_ARG
+    assert call(lens.data_ptr(), rule=5) == ds.DS_ERR_INVALID_ARG
 
 
 # ------------------------------------------------------ offloaded caches
