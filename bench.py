@@ -18,6 +18,7 @@ Rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -225,6 +226,29 @@ def _dev(x: np.ndarray, dtype: str, dev):
     return torch.from_numpy(np.ascontiguousarray(x)).to(dev)
 
 
+def rotation(wl, dev, kind: str, out_esz: int):
+    """How many independent layer instances the timed steps cycle through.
+    'rotate': enough copies that their working sets together exceed twice the
+    L2, so no step finds its inputs in L2 from an earlier step (a workload
+    whose own working set is that large needs one); tiny workloads, where 16
+    copies would still fit, fall back to 'flush'."""
+    import math
+
+    import torch
+    if kind != "rotate":
+        return kind, 1
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    ws = algorithmic_bytes(wl, out_esz)["total"]
+    r = max(1, math.ceil(2 * l2 / ws))
+    if r > 16:
+        return "flush", 1
+    return "rotate", r
+
+
+def _clone_state(st):
+    return {n: (t.clone() if t is not None and hasattr(t, "clone") and n != "idx" else t) for n, t in st.items()}
+
+
 def run_ours(args, wl, rank, local_rank, world):
     import torch
 
@@ -233,17 +257,21 @@ def run_ours(args, wl, rank, local_rank, world):
     ds.build()
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    st = build_state(wl, dev, rank)
-    q, k, v, idx, lab, sc, ze = (st[n] for n in ("q", "k", "v", "idx", "lab", "sc", "ze"))
+    out_dtype = torch.bfloat16 if wl.kv_dtype == "bf16" else torch.float32
+    timing, R = rotation(wl, dev, args.timing, 2 if out_dtype == torch.bfloat16 else 4)
+    st0 = build_state(wl, dev, rank)
+    states = [st0] + [_clone_state(st0) for _ in range(R - 1)]
+    for st in states:
+        st["out"] = torch.empty((wl.b, wl.hq, wl.d), dtype=out_dtype, device=dev)
+    q, k, v, idx, lab, sc, ze, out = (st0[n] for n in ("q", "k", "v", "idx", "lab", "sc", "ze", "out"))
     pos = wl.s - 1
-    out = torch.empty((wl.b, wl.hq, wl.d), dtype=torch.bfloat16 if wl.kv_dtype == "bf16" else torch.float32,
-                      device=dev)
     flush = L2Flush(dev, args.flush)
     stream = torch.cuda.Stream(device=dev)
 
     # prefill: label cache for the first s-1 tokens (timed separately, after
     # one untimed call that loads the kernel)
-    ds.build_label_cache(k, idx, pos, lab, sc, ze)
+    for st in states:
+        ds.build_label_cache(st["k"], st["idx"], pos, st["lab"], st["sc"], st["ze"])
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     flush()
@@ -253,44 +281,65 @@ def run_ours(args, wl, rank, local_rank, world):
     torch.cuda.synchronize()
     prefill_ms = e0.elapsed_time(e1)
 
-    def step():
+    def step_of(st):
         # one launch: label row of token s-1 (ds_append_label's work) + sparse decode
-        ds.decode_step(q, k, v, lab, idx, wl.s, wl.topk, lscale=sc, lzero=ze, out=out)
+        return lambda: ds.decode_step(st["q"], st["k"], st["v"], st["lab"], st["idx"], wl.s, wl.topk,
+                                      lscale=st["sc"], lzero=st["ze"], out=st["out"])
 
-    with torch.cuda.stream(stream):
-        for _ in range(3):  # set kernel attributes before capture
-            step()
-    stream.synchronize()
-    g_step = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_step, stream=stream):
-        step()
+    graphs = []
+    for st in states:
+        fn = step_of(st)
+        with torch.cuda.stream(stream):
+            for _ in range(3):  # set kernel attributes before capture
+                fn()
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        graphs.append(g)
 
-    def one_step(evs=None):
-        flush()  # untimed: evicts L2 (the step's inputs could otherwise stay in the 126 MB L2)
+    def one_step(i, evs=None):
+        if timing == "flush":
+            flush()  # untimed: evicts L2 (the step's inputs could otherwise stay in the 126 MB L2)
         if evs:
             evs[0].record()
-        g_step.replay()
+        graphs[i % R].replay()
         if evs:
             evs[1].record()
 
     with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            one_step()
+        for i in range(args.warmup):
+            one_step(i)
     torch.cuda.synchronize()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     sampler = ClockSampler(local_rank)
     barrier()
     torch.cuda.synchronize()
-    with sampler:
-        wall0 = time.perf_counter()
-        with torch.cuda.stream(stream):
-            for i in range(args.steps):
-                one_step(evs[i])
-        torch.cuda.synchronize()
-        wall1 = time.perf_counter()
+    if timing == "flush":
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        with sampler:
+            wall0 = time.perf_counter()
+            with torch.cuda.stream(stream):
+                for i in range(args.steps):
+                    one_step(i, evs[i])
+            torch.cuda.synchronize()
+            wall1 = time.perf_counter()
+        step_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    else:
+        # back to back, cycling through the R layer instances; one event pair
+        # around the K steps on the launching stream
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with sampler:
+            wall0 = time.perf_counter()
+            with torch.cuda.stream(stream):
+                t0.record()
+                for i in range(args.steps):
+                    one_step(args.warmup + i)
+                t1.record()
+            torch.cuda.synchronize()
+            wall1 = time.perf_counter()
+        step_ms = [t0.elapsed_time(t1) / args.steps] * args.steps
     barrier()
-    step_ms = [e[0].elapsed_time(e[1]) for e in evs]
     total_s = sum(step_ms) / 1e3
     max_s = reduce_max(total_s, dev)
 
@@ -303,22 +352,38 @@ def run_ours(args, wl, rank, local_rank, world):
     hq.copy_(q.cpu()); hk.copy_(k[:, :, pos].cpu()); hv.copy_(v[:, :, pos].cpu())
     hout = torch.empty_like(out, device="cpu").pin_memory()
     dq, dk, dv = torch.empty_like(q), torch.empty_like(hk, device=dev), torch.empty_like(hv, device=dev)
+
+    def e2e_step(i):
+        st = states[i % R]
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        st["k"][:, :, pos].copy_(dk)
+        st["v"][:, :, pos].copy_(dv)
+        ds.decode_step(dq, st["k"], st["v"], st["lab"], st["idx"], wl.s, wl.topk, lscale=st["sc"],
+                       lzero=st["ze"], out=st["out"])
+        hout.copy_(st["out"], non_blocking=True)
+
     e2e_ms = []
     with torch.cuda.stream(stream):
-        for i in range(args.warmup + args.steps):
-            flush()
+        if timing == "flush":
+            for i in range(args.warmup + args.steps):
+                flush()
+                a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                e2e_step(i)
+                b_.record()
+                if i >= args.warmup:
+                    e2e_ms.append((a, b_))
+        else:
+            for i in range(args.warmup):
+                e2e_step(i)
             a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
-            dq.copy_(hq, non_blocking=True)
-            dk.copy_(hk, non_blocking=True)
-            dv.copy_(hv, non_blocking=True)
-            k[:, :, pos].copy_(dk)
-            v[:, :, pos].copy_(dv)
-            ds.decode_step(dq, k, v, lab, idx, wl.s, wl.topk, lscale=sc, lzero=ze, out=out)
-            hout.copy_(out, non_blocking=True)
+            for i in range(args.steps):
+                e2e_step(args.warmup + i)
             b_.record()
-            if i >= args.warmup:
-                e2e_ms.append((a, b_))
+            e2e_ms.append((a, b_))
     torch.cuda.synchronize()
     e2e_s = sum(a.elapsed_time(b_) for a, b_ in e2e_ms) / 1e3
     e2e_max = reduce_max(e2e_s, dev)
@@ -326,10 +391,10 @@ def run_ours(args, wl, rank, local_rank, world):
     d2h = out.numel() * out.element_size()
 
     # dense baseline on the same cache: our dense kernel and torch SDPA
-    dense_ms, sdpa_ms = dense_baselines(wl, q, k, v, out, flush, stream)
+    dense_ms, sdpa_ms = dense_baselines(wl, q, k, v, out, flush if timing == "flush" else None, stream)
     offload = offload_timing(wl, q, k, v, idx, lab, sc, ze, out, flush, stream) if args.offload else None
 
-    res = dict(step_ms=step_ms, total_s=total_s, max_s=max_s,
+    res = dict(step_ms=step_ms, total_s=total_s, max_s=max_s, timing=timing, rotate=R,
                wall_s=wall1 - wall0, e2e_s=e2e_max, h2d=h2d, d2h=d2h, prefill_ms=prefill_ms,
                clocks=sampler.summary(), dense_ms=dense_ms, sdpa_ms=sdpa_ms, offload=offload,
                plan=ds.plan(wl.b, wl.hq, wl.hkv, wl.s, wl.d, wl.c, wl.topk,
@@ -341,9 +406,13 @@ def run_ours(args, wl, rank, local_rank, world):
 
 
 class L2Flush:
-    """Evicts L2 between timed steps by writing FLUSH_BYTES (> the 126 MB L2):
-    'copy' = a device-to-device copy of FLUSH_BYTES/2 (copy engine, no SM
-    kernel runs between steps), 'fill' = an elementwise fill kernel."""
+    """Evicts L2 between timed steps by writing FLUSH_BYTES (> the 126 MB L2).
+    'write_read' (default) = a fill kernel over FLUSH_BYTES, then a reduction
+    that reads another FLUSH_BYTES: the written lines are written back to HBM
+    before the timed region instead of during the step, and L2 is left holding
+    only clean lines of the flush buffer. 'copy' = a device-to-device copy of
+    FLUSH_BYTES/2; 'fill' = the fill kernel alone (both leave up to an L2 of
+    dirty flush data, whose write-back the next step then pays for)."""
 
     def __init__(self, dev, kind: str):
         import torch
@@ -353,15 +422,22 @@ class L2Flush:
             self.dst = torch.empty_like(self.src)
         else:
             self.buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+            if kind == "write_read":
+                self.rd = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
     def __call__(self):
         if self.kind == "copy":
             self.dst.copy_(self.src)
         else:
             self.buf.zero_()
+            if self.kind == "write_read":
+                self.rd.sum()
 
 
 def dense_baselines(wl, q, k, v, out, flush, stream, reps=20):
+    """Dense decode over the same cache (ds_dense_decode and torch SDPA), in
+    ms per call: with `flush`, the median of single calls after an L2 flush;
+    without, the mean of back-to-back calls (their K+V exceed the L2)."""
     import torch
     import torch.nn.functional as F
 
@@ -372,14 +448,23 @@ def dense_baselines(wl, q, k, v, out, flush, stream, reps=20):
             for _ in range(3):
                 fn()
             ts = []
-            for _ in range(reps):
-                flush()
+            if flush is None:
                 a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record()
-                fn()
+                for _ in range(reps):
+                    fn()
                 b_.record()
-                ts.append((a, b_))
+            else:
+                for _ in range(reps):
+                    flush()
+                    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a.record()
+                    fn()
+                    b_.record()
+                    ts.append((a, b_))
         torch.cuda.synchronize()
+        if flush is None:
+            return a.elapsed_time(b_) / reps
         return statistics.median(a.elapsed_time(b_) for a, b_ in ts)
 
     dense_ms = timed(lambda: ds.dense_decode(q, k, v, wl.s, out=out))
@@ -497,7 +582,7 @@ def run_reference(args, wl):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": workload_config(wl, None),
+            "data": "synthetic", "config": {**workload_config(wl, None), "l2": "not applicable (CPU oracle)"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
@@ -506,7 +591,7 @@ def run_reference(args, wl):
 def workload_config(wl, plan):
     cfg = {"workload": wl.name, "batch": wl.b, "q_heads": wl.hq, "kv_heads": wl.hkv, "head_dim": wl.d,
            "seq_len": wl.s, "heavy_channels": wl.c, "label": wl.label_dtype, "topk": wl.topk,
-           "kv_dtype": wl.kv_dtype, "l2": "flushed before every timed step"}
+           "kv_dtype": wl.kv_dtype}
     if plan:
         cfg["cluster_ctas"], cfg["tokens_per_cta"], cfg["smem_bytes"] = plan
     return cfg
@@ -523,12 +608,21 @@ def main():
     ap.add_argument("--config", type=int, default=1, help="workload index (0-4)")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=8, help="rows per reference-arm step")
+    ap.add_argument("--label", default=None, choices=["f32", "bf16", "int4"],
+                    help="override the workload's label cache dtype (measurement variants)")
     ap.add_argument("--offload", action="store_true",
                     help="also time the step with the K/V caches in pinned host memory")
-    ap.add_argument("--flush", default="copy", choices=["copy", "fill"],
-                    help="L2 eviction between timed steps: D2D copy or fill kernel")
+    ap.add_argument("--timing", default="rotate", choices=["rotate", "flush"],
+                    help="rotate: back-to-back steps cycling through enough layer instances that the "
+                         "inputs exceed the L2; flush: one step per event pair after an L2 flush")
+    ap.add_argument("--flush", default="write_read", choices=["write_read", "copy", "fill"],
+                    help="L2 eviction between timed steps: fill then read (default), D2D copy, or fill kernel")
     args = ap.parse_args()
     wl = synth.workload(args.config)
+    if args.label and args.label != wl.label_dtype:
+        if args.label != "int4" and args.label != wl.kv_dtype:
+            raise SystemExit("an fp label cache has the key cache's dtype")
+        wl = dataclasses.replace(wl, label_dtype=args.label, name=f"{wl.name}, {args.label} label")
     rank, local_rank, world = dist_env()
 
     if args.impl == "reference":
@@ -558,6 +652,17 @@ def main():
             dist.destroy_process_group()
 
 
+def l2_note(args, r) -> str:
+    if r["timing"] == "rotate":
+        return (f"inputs larger than L2: the {args.steps} timed steps run back to back, cycling through "
+                f"{r['rotate']} independent layer instances (own q, K, V, label cache and output) whose "
+                f"working sets together exceed twice the L2; one event pair around the K steps")
+    return (f"flushed before every timed step: {FLUSH_BYTES >> 20} MiB written by "
+            + ("a device-to-device copy" if args.flush == "copy" else "a fill kernel")
+            + (f", then {FLUSH_BYTES >> 20} MiB read (flush data written back before the step)"
+               if args.flush == "write_read" else ""))
+
+
 def report(args, wl, r, world):
     ab = algorithmic_bytes(wl, r["out_esz"])
     peaks = measured_peaks()
@@ -578,13 +683,13 @@ def report(args, wl, r, world):
         "scaling": "weak", "vs_baseline": None, "dtype": wl.kv_dtype, "data": "synthetic (seeded N(0,1) "
         "Q/K/V with planted outlier channels)",
         "config": {**workload_config(wl, r["plan"]), "parallelism": f"dp{world} (independent layers per rank)",
-                   "l2": f"flushed before every timed step: {FLUSH_BYTES >> 20} MiB written by "
-                         + ("a device-to-device copy" if args.flush == "copy" else "a fill kernel")},
+                   "l2": l2_note(args, r)},
         "hbm_gbs": achieved, "pct_of_nominal_hbm": 100 * achieved / NOMINAL_HBM_GBS,
         "pct_of_measured_hbm": 100 * achieved / peaks["hbm_gbs"],
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"],
-                     "traffic": recorded_traffic(args.config), "kernel": "ds_decode_kernel",
+                     "traffic": (recorded_traffic(args.config)
+                                 if wl.label_dtype == synth.workload(args.config).label_dtype else None), "kernel": "ds_decode_kernel",
                      "algorithmic_bytes_per_launch": ab["total"], "avg_launch_us": dec_avg_s * 1e6},
         "step_us": dec_avg_s * 1e6,
         "cpu_baseline": cpu,

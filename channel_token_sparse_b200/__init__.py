@@ -34,6 +34,10 @@ SIGNATURES = {
     "ds_calibrate_workspace_size": (_i, [_i, _i, _i, _i, _i, _i, C.POINTER(_sz)]),
     "ds_calibrate_channels": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp]),
     "ds_calibrate_channels_noalloc": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "ds_build_label_cache_paged": (_i, [_vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _i, _vp,
+                                        _vp, _vp]),
+    "ds_decode_step_paged": (_i, [_vp, _vp, _vp, _i, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _i, _i, _i,
+                                  _i, _i, _i, _i, _i, _i, _i, _f, _vp, _i, _vp, _vp, _vp]),
     "ds_calibrate_channels_criterion": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp,
                                              _vp, _sz, _vp]),
     "ds_build_label_cache": (_i, [_vp, _i, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _vp]),
@@ -329,6 +333,49 @@ def decode_step_varlen(q, k, v, label, idx, seq_lens, s_max: int, topk: int, lsc
                                        b, hq, hkv, s_max, s_cap, d, c, topk,
                                        float(sm_scale), _ptr(out), odt, _ptr(sel_out), _ptr(score_out),
                                        _stream(stream)))
+    return out
+
+
+def build_label_cache_paged(k_pool, idx, block_table, s: int, label, lscale=None, lzero=None, stream=None):
+    """Fill label rows [0, s) (label [B, Hkv, S_cap, ...]) from a paged key
+    pool k_pool [num_blocks, Hkv, page, D] through block_table [B, max_blocks]."""
+    _need_cuda_or_pinned(k_pool)
+    _need_cuda(idx, block_table, label, lscale, lzero)
+    num_blocks, hkv, page, d = k_pool.shape
+    b, max_blocks = block_table.shape
+    s_cap = label.shape[2]
+    c = idx.shape[1]
+    kdt = _kv_dtype(k_pool)
+    _check(lib().ds_build_label_cache_paged(_ptr_kv(k_pool), kdt, _ptr(idx), _ptr(block_table), max_blocks, page,
+                                            num_blocks, b, hkv, s, s_cap, d, c, _ptr(label),
+                                            _label_args(label, lscale, lzero, kdt), _ptr(lscale), _ptr(lzero),
+                                            _stream(stream)))
+
+
+def decode_step_paged(q, k_pool, v_pool, label, idx, block_table, s_max: int, topk: int, seq_lens=None,
+                      lscale=None, lzero=None, out=None, out_dtype=None, sm_scale: float = 0.0, sel_out=None,
+                      score_out=None, sparse_threshold: int = 0, fallback: int = DS_FALLBACK_PER_ENTRY,
+                      stream=None):
+    """decode_step(_varlen) over paged pools k_pool/v_pool [num_blocks, Hkv,
+    page, D] with block_table [B, max_blocks]; returns out [B, Hq, D]."""
+    torch = _torch()
+    _need_cuda_or_pinned(k_pool, v_pool)
+    _need_cuda(q, label, idx, block_table, seq_lens, lscale, lzero, out, sel_out, score_out)
+    b, hq, d = q.shape
+    num_blocks, hkv, page, _ = k_pool.shape
+    max_blocks = block_table.shape[1]
+    s_cap = label.shape[2]
+    c = idx.shape[1]
+    kdt = _kv_dtype(k_pool)
+    if out is None:
+        out = torch.empty((b, hq, d), dtype=out_dtype or torch.float32, device=q.device)
+    odt = DS_F32 if out.dtype == torch.float32 else DS_BF16
+    _check(lib().ds_decode_step_paged(_ptr(q), _ptr_kv(k_pool), _ptr_kv(v_pool), kdt, _ptr(label),
+                                      _label_args(label, lscale, lzero, kdt), _ptr(lscale), _ptr(lzero),
+                                      _ptr(idx), _ptr(block_table), max_blocks, page, num_blocks, _ptr(seq_lens),
+                                      int(sparse_threshold), int(fallback), b, hq, hkv, s_max, s_cap, d, c, topk,
+                                      float(sm_scale), _ptr(out), odt, _ptr(sel_out), _ptr(score_out),
+                                      _stream(stream)))
     return out
 
 

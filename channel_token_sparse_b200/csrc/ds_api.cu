@@ -195,16 +195,52 @@ ds_status check_label(ds_dtype kdt, ds_dtype label_dt, int c, int d, const void*
     return DS_OK;
 }
 
+// Paged K/V: a block table [b, max_blocks] of block ids into pools
+// [num_blocks, hkv, page_size, d].
+struct Paged {
+    const int32_t* bt = nullptr;
+    int max_blocks = 0, page_size = 0, num_blocks = 0;
+};
+
+int log2_exact(int x) {
+    int l = 0;
+    while ((1 << l) < x) ++l;
+    return (1 << l) == x ? l : -1;
+}
+
+ds_status check_paged(const Paged& pg, int s_max, int hkv, int d) {
+    if (!pg.bt) return fail(DS_ERR_INVALID_ARG, "block_table is NULL");
+    if (reinterpret_cast<uintptr_t>(pg.bt) % 4) return fail(DS_ERR_INVALID_ARG, "block_table not 4-byte aligned");
+    if (pg.page_size < 1 || pg.page_size > (1 << 16) || log2_exact(pg.page_size) < 0)
+        return fail(DS_ERR_INVALID_ARG, "page_size %d must be a power of two in [1, 65536]", pg.page_size);
+    if (pg.num_blocks < 1 || pg.max_blocks < 1) return fail(DS_ERR_INVALID_ARG, "num_blocks and max_blocks must be >= 1");
+    if ((long long)pg.max_blocks * pg.page_size < s_max)
+        return fail(DS_ERR_INVALID_ARG, "max_blocks * page_size (%lld) < tokens (%d)",
+                    (long long)pg.max_blocks * pg.page_size, s_max);
+    if ((long long)pg.num_blocks * hkv * pg.page_size >= (1ll << 32))
+        return fail(DS_ERR_UNSUPPORTED, "pool too large (rows must fit 32 bits)");
+    if ((long long)pg.num_blocks * hkv * pg.page_size * d >= (1ll << 40))
+        return fail(DS_ERR_UNSUPPORTED, "pool too large");
+    return DS_OK;
+}
+
 ds_status run_label(const void* k, ds_dtype kdt, const int32_t* idx, int b, int hkv, int t_begin,
                     int t_end, int s_cap, int d, int c, void* label, ds_dtype label_dt,
-                    uint16_t* lscale, uint16_t* lzero, cudaStream_t st) {
+                    uint16_t* lscale, uint16_t* lzero, cudaStream_t st, const Paged* pg = nullptr) {
     ds_status r = check_common(b, hkv, hkv, t_end, s_cap, d, kdt);
     if (r != DS_OK) return r;
+    if (pg && (r = check_paged(*pg, t_end, hkv, d)) != DS_OK) return r;
     if ((r = check_label(kdt, label_dt, c, d, label, lscale, lzero)) != DS_OK) return r;
     if (!k || !idx) return fail(DS_ERR_INVALID_ARG, "k or idx is NULL");
     if (!aligned16(k) || !aligned16(idx)) return fail(DS_ERR_INVALID_ARG, "k/idx not 16-byte aligned");
     ds::LabelArgs a{k, kdt == DS_BF16, label_dt == DS_INT4, idx, b, hkv, t_begin, t_end, s_cap, d, c,
                     label, lscale, lzero};
+    if (pg) {
+        a.block_table = pg->bt;
+        a.max_blocks = pg->max_blocks;
+        a.page_shift = log2_exact(pg->page_size);
+        a.num_blocks = pg->num_blocks;
+    }
     cudaError_t e = ds::launch_label(a, st);
     if (e != cudaSuccess) return cuda_fail(e, "label launch");
     return DS_OK;
@@ -352,9 +388,10 @@ ds_status sparse_decode_impl(const void* q, const void* k, const void* v, ds_dty
                              const int32_t* idx, int b, int hq, int hkv, int s, int s_cap, int d, int c,
                              int topk, float sm_scale, void* out, ds_dtype out_dt, int32_t* sel_out,
                              float* score_out, bool append, const int32_t* seq_lens, int threshold,
-                             int batch_rule, cudaStream_t stream) {
+                             int batch_rule, cudaStream_t stream, const Paged* pg = nullptr) {
     ds_status r = check_common(b, hq, hkv, s, s_cap, d, kvdt);
     if (r != DS_OK) return r;
+    if (pg && (r = check_paged(*pg, s, hkv, d)) != DS_OK) return r;
     if ((r = check_label(kvdt, label_dt, c, d, label, lscale, lzero)) != DS_OK) return r;
     if (topk < 1) return fail(DS_ERR_INVALID_ARG, "topk must be >= 1");
     if (!q || !k || !v || !idx || !out) return fail(DS_ERR_INVALID_ARG, "NULL pointer");
@@ -380,6 +417,12 @@ ds_status sparse_decode_impl(const void* q, const void* k, const void* v, ds_dty
     p.nb = b;
     p.threshold = threshold;
     p.batch_rule = batch_rule;
+    if (pg) {
+        p.block_table = pg->bt;
+        p.max_blocks = pg->max_blocks;
+        p.page_shift = log2_exact(pg->page_size);
+        p.num_blocks = pg->num_blocks;
+    }
     p.out = out; p.sel_out = sel_out; p.score_out = score_out;
     p.hkv = hkv; p.G = G; p.s = s; p.s_cap = s_cap; p.topk = topk;
     p.chunk = pl.chunk; p.lay_chunk = pl.lay_chunk; p.per = pl.per;
@@ -429,6 +472,32 @@ ds_status ds_decode_step_varlen(const void* q, const void* k, const void* v, ds_
     return sparse_decode_impl(q, k, v, kvdt, label, label_dt, lscale, lzero, idx, b, hq, hkv, s_max, s_cap, d, c,
                               topk, sm_scale, out, out_dt, sel_out, score_out, true, seq_lens, sparse_threshold,
                               fallback == DS_FALLBACK_BATCH ? 1 : 0, stream);
+}
+
+ds_status ds_build_label_cache_paged(const void* k_pool, ds_dtype kdt, const int32_t* idx,
+                                     const int32_t* block_table, int max_blocks, int page_size, int num_blocks,
+                                     int b, int hkv, int s, int s_cap, int d, int c, void* label,
+                                     ds_dtype label_dt, uint16_t* lscale, uint16_t* lzero, cudaStream_t stream) {
+    Paged pg;
+    pg.bt = block_table; pg.max_blocks = max_blocks; pg.page_size = page_size; pg.num_blocks = num_blocks;
+    return run_label(k_pool, kdt, idx, b, hkv, 0, s, s_cap, d, c, label, label_dt, lscale, lzero, stream, &pg);
+}
+
+ds_status ds_decode_step_paged(const void* q, const void* k_pool, const void* v_pool, ds_dtype kvdt, void* label,
+                               ds_dtype label_dt, uint16_t* lscale, uint16_t* lzero, const int32_t* idx,
+                               const int32_t* block_table, int max_blocks, int page_size, int num_blocks,
+                               const int32_t* seq_lens, int sparse_threshold, ds_fallback fallback, int b,
+                               int hq, int hkv, int s_max, int s_cap, int d, int c, int topk, float sm_scale,
+                               void* out, ds_dtype out_dt, int32_t* sel_out, float* score_out,
+                               cudaStream_t stream) {
+    if (sparse_threshold < 0) return fail(DS_ERR_INVALID_ARG, "sparse_threshold (%d) < 0", sparse_threshold);
+    if (fallback != DS_FALLBACK_PER_ENTRY && fallback != DS_FALLBACK_BATCH)
+        return fail(DS_ERR_INVALID_ARG, "unknown fallback rule %d", (int)fallback);
+    Paged pg;
+    pg.bt = block_table; pg.max_blocks = max_blocks; pg.page_size = page_size; pg.num_blocks = num_blocks;
+    return sparse_decode_impl(q, k_pool, v_pool, kvdt, label, label_dt, lscale, lzero, idx, b, hq, hkv, s_max, s_cap,
+                              d, c, topk, sm_scale, out, out_dt, sel_out, score_out, true, seq_lens,
+                              sparse_threshold, fallback == DS_FALLBACK_BATCH ? 1 : 0, stream, &pg);
 }
 
 ds_status ds_dense_decode(const void* q, const void* k, const void* v, ds_dtype kvdt, int b, int hq,

@@ -66,7 +66,21 @@ struct DecodeParams {
     // attends all its tokens when the longest is shorter than `threshold` or
     // the shortest is shorter than topk)
     int nb, threshold, batch_rule;
+    // paged K/V (null block_table: K/V are [b, hkv, s_cap, d]): K/V pools are
+    // [num_blocks, hkv, 1 << page_shift, d] and token t of batch entry b is
+    // row t & (page - 1) of block block_table[b * max_blocks + (t >> page_shift)]
+    const int32_t* block_table;
+    int max_blocks, page_shift, num_blocks;
 };
+
+// Row (in units of d elements) of token t of (b, g) in the K/V caches, dense
+// or paged; block ids are clamped into the pool.
+__device__ __forceinline__ size_t kv_row_of(const DecodeParams& p, int b, int g, size_t row_tok, int t) {
+    if (!p.block_table) return row_tok + (size_t)t;
+    int blk = __ldg(p.block_table + (size_t)b * p.max_blocks + (t >> p.page_shift));
+    blk = min(max(blk, 0), p.num_blocks - 1);
+    return (((size_t)blk * p.hkv + g) << p.page_shift) + (size_t)(t & ((1 << p.page_shift) - 1));
+}
 
 // Shared-memory carve-up (bytes), identical on host and device.
 struct DecodeSmem {
@@ -295,8 +309,8 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     constexpr int kKRowVecs = D * E::kBytes / 16;   // 16-byte pieces of a key row
     uint4 kv_app = make_uint4(0u, 0u, 0u, 0u);
     if (app_i >= 0 && tid < kKRowVecs)
-        kv_app = ldg_stream16(reinterpret_cast<const uint8_t*>(p.k) + ((row_tok + (size_t)(s - 1)) * D) * E::kBytes +
-                              tid * 16);
+        kv_app = ldg_stream16(reinterpret_cast<const uint8_t*>(p.k) +
+                              (kv_row_of(p, row / p.hkv, g, row_tok, s - 1) * D) * E::kBytes + tid * 16);
 
     // fp label rows stream through a kLabStages-deep shared-memory ring with
     // cp.async (no registers held while in flight): in stage j, thread tid
@@ -464,8 +478,8 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
 
     // [phase] 2
     // --------------------------------------------------------------- step 3a
-    const TKV* kb = reinterpret_cast<const TKV*>(p.k) + row_tok * D;
-    const TKV* vb = reinterpret_cast<const TKV*>(p.v) + row_tok * D;
+    const TKV* kb = reinterpret_cast<const TKV*>(p.k);   // rows addressed by att_row()
+    const TKV* vb = reinterpret_cast<const TKV*>(p.v);
     constexpr int RB = D * E::kBytes;              // bytes of one K or V row
     int T16 = 0, Tlo = 0, r_tie = 0;
     bool refine = false;
@@ -723,249 +737,268 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     // [phase] 6
     // --------------------------------------------------------------- step 3b
     const int n_att = select_all ? n_loc : max(0, min(p.per, k_eff - rank * p.per));
-    auto att_token = [&](int j) -> int { return select_all ? t0 + j : sel_list[j]; };
+    // paged K/V: this CTA's selected tokens become pool rows first (one
+    // table lookup per token, all in flight together)
+    uint32_t* sel_rows = reinterpret_cast<uint32_t*>(sel_list);
+    if (p.block_table && !select_all) {
+        for (int j = tid; j < n_att; j += kNT)
+            sel_rows[j] = (uint32_t)kv_row_of(p, row / p.hkv, g, row_tok, sel_list[j]);
+        __syncthreads();
+    }
     float* wp_out = nullptr;  // this warp's partial (m, l, o) per head, [GT][D + 2]
     auto write_out = [&](int h, int d, float res) {
         const size_t oidx = (size_t)row * G * D + (size_t)h * D + d;
         if (p.out_bf16) reinterpret_cast<uint16_t*>(p.out)[oidx] = f32_to_bf16_bits(res);
         else reinterpret_cast<float*>(p.out)[oidx] = res;
     };
-    if constexpr (E::kBytes == 2) {
-        // bf16 K/V: tensor cores (mma.sync, fp32 accumulate) on 8-token tiles.
-        //   Z  = Q K^T   m16n8k16: rows = the group's heads (padded to 16),
-        //                cols = 8 tokens, k = 16 dims per step
-        //   O^T += V^T P^T  m16n8k8: rows = 16 dims, cols = heads, k = 8 tokens
-        // so the softmax probabilities of a head (a row of Z's accumulator)
-        // are already laid out as the B operand of the second product. P is
-        // split into bf16 hi + lo parts (two products), keeping ~2^-17 of
-        // relative precision. Rows are staged with cp.async into a per-warp
-        // ring; 16-byte chunks are XOR-swizzled by token so that ldmatrix reads
-        // are bank-conflict free.
-        constexpr int TB8 = 8;
-        constexpr int kChunks = RB / 16;           // 16-byte chunks per row
-        constexpr int kStageBytes = 2 * TB8 * RB;
-        const int stages = p.att_stages;
-        uint8_t* ring = smem + L.region + wid * att_ring_bytes(RB, 2, stages);
-        const int nb = n_att > wid * TB8 ? (n_att - wid * TB8 + kNW * TB8 - 1) / (kNW * TB8) : 0;
-        auto issue_stage = [&](int bi) {
-            const int bt0 = (wid + bi * kNW) * TB8;
-            uint8_t* st = ring + (bi % stages) * kStageBytes;
-#pragma unroll
-            for (int pc = lane; pc < 2 * TB8 * kChunks; pc += 32) {
-                const int r = pc / kChunks, c = pc - r * kChunks;
-                const int u = r & (TB8 - 1);
-                const bool ok = bt0 + u < n_att;
-                const TKV* base = r < TB8 ? kb : vb;
-                const TKV* src = ok ? base + (size_t)att_token(bt0 + u) * D : base;
-                // rows of tokens past the end are zero-filled (their p is 0, and 0 * garbage could be NaN)
-                cp_async16_zfill(st + r * RB + ((c ^ u) << 4), reinterpret_cast<const uint8_t*>(src) + (c << 4), ok);
+    // The attention phase, instantiated once per K/V addressing (dense
+    // caches, or paged pools through the block table) so that the row lookup
+    // adds no branch to the copy loops. att_row(j) is the K/V row (units of d
+    // elements) of the j-th token this CTA attends.
+    auto attend = [&](auto att_row) {
+        if constexpr (E::kBytes == 2) {
+            // bf16 K/V: tensor cores (mma.sync, fp32 accumulate) on 8-token tiles.
+            //   Z  = Q K^T   m16n8k16: rows = the group's heads (padded to 16),
+            //                cols = 8 tokens, k = 16 dims per step
+            //   O^T += V^T P^T  m16n8k8: rows = 16 dims, cols = heads, k = 8 tokens
+            // so the softmax probabilities of a head (a row of Z's accumulator)
+            // are already laid out as the B operand of the second product. P is
+            // split into bf16 hi + lo parts (two products), keeping ~2^-17 of
+            // relative precision. Rows are staged with cp.async into a per-warp
+            // ring; 16-byte chunks are XOR-swizzled by token so that ldmatrix reads
+            // are bank-conflict free.
+            constexpr int TB8 = 8;
+            constexpr int kChunks = RB / 16;           // 16-byte chunks per row
+            constexpr int kStageBytes = 2 * TB8 * RB;
+            const int stages = p.att_stages;
+            uint8_t* ring = smem + L.region + wid * att_ring_bytes(RB, 2, stages);
+            const int nb = n_att > wid * TB8 ? (n_att - wid * TB8 + kNW * TB8 - 1) / (kNW * TB8) : 0;
+            auto issue_stage = [&](int bi) {
+                const int bt0 = (wid + bi * kNW) * TB8;
+                uint8_t* st = ring + (bi % stages) * kStageBytes;
+    #pragma unroll
+                for (int pc = lane; pc < 2 * TB8 * kChunks; pc += 32) {
+                    const int r = pc / kChunks, c = pc - r * kChunks;
+                    const int u = r & (TB8 - 1);
+                    const bool ok = bt0 + u < n_att;
+                    const TKV* base = r < TB8 ? kb : vb;
+                    const TKV* src = ok ? base + att_row(bt0 + u) * D : base;
+                    // rows of tokens past the end are zero-filled (their p is 0, and 0 * garbage could be NaN)
+                    cp_async16_zfill(st + r * RB + ((c ^ u) << 4), reinterpret_cast<const uint8_t*>(src) + (c << 4), ok);
+                }
+            };
+            for (int bi = 0; bi < stages - 1; ++bi) {
+                if (bi < nb) issue_stage(bi);
+                cp_async_commit();
             }
-        };
-        for (int bi = 0; bi < stages - 1; ++bi) {
-            if (bi < nb) issue_stage(bi);
-            cp_async_commit();
-        }
-        // Q fragments (A operand, rows = heads): bf16 pairs, exact (q is bf16),
-        // kept in shared memory ([D/16 steps][32 lanes][2 words]) to spare registers
-        const int hr = lane >> 2, kc = (lane & 3) * 2;
-        const uint2* qa = reinterpret_cast<const uint2*>(smem + L.qa);
-        float o[D / 16][4];
-#pragma unroll
-        for (int i = 0; i < D / 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-        float m_run = -INFINITY, l_run = 0.f;  // for head hr (row of Z)
-        // [phase] 21
-#pragma unroll 1
-        for (int bi = 0; bi < nb; ++bi) {
-            if (bi + stages - 1 < nb) issue_stage(bi + stages - 1);
-            cp_async_commit();
-            if (stages == 3) cp_async_wait<2>();
-            else cp_async_wait<1>();
+            // Q fragments (A operand, rows = heads): bf16 pairs, exact (q is bf16),
+            // kept in shared memory ([D/16 steps][32 lanes][2 words]) to spare registers
+            const int hr = lane >> 2, kc = (lane & 3) * 2;
+            const uint2* qa = reinterpret_cast<const uint2*>(smem + L.qa);
+            float o[D / 16][4];
+    #pragma unroll
+            for (int i = 0; i < D / 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+            float m_run = -INFINITY, l_run = 0.f;  // for head hr (row of Z)
+            // [phase] 21
+    #pragma unroll 1
+            for (int bi = 0; bi < nb; ++bi) {
+                if (bi + stages - 1 < nb) issue_stage(bi + stages - 1);
+                cp_async_commit();
+                if (stages == 3) cp_async_wait<2>();
+                else cp_async_wait<1>();
+                __syncwarp();
+                const uint8_t* st = ring + (bi % stages) * kStageBytes;
+                const int bt0 = (wid + bi * kNW) * TB8;
+                // Z = Q K^T over D in 16-dim steps; one ldmatrix.x4 covers 32 dims
+                float z[4] = {0.f, 0.f, 0.f, 0.f};
+                const int mr = lane & 7, mi = lane >> 3;  // ldmatrix: row (token) and matrix index
+    #pragma unroll
+                for (int c4 = 0; c4 < D / 32; ++c4) {
+                    uint32_t b[4];
+                    ldmatrix_x4(b, st + mr * RB + (((4 * c4 + mi) ^ mr) << 4));
+                    const uint2 q0 = qa[(2 * c4) * 32 + lane], q1 = qa[(2 * c4 + 1) * 32 + lane];
+                    mma_bf16_16816(z, q0.x, 0u, q0.y, 0u, b[0], b[1]);
+                    mma_bf16_16816(z, q1.x, 0u, q1.y, 0u, b[2], b[3]);
+                }
+                // online softmax for head hr over tokens kc, kc + 1 of the tile
+                const bool ok0 = bt0 + kc < n_att, ok1 = bt0 + kc + 1 < n_att;
+                const float z0 = ok0 ? z[0] * p.qscale : -INFINITY;
+                const float z1 = ok1 ? z[1] * p.qscale : -INFINITY;
+                float mx = fmaxf(z0, z1);
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                const float m_new = fmaxf(m_run, mx);
+                const float corr = exp2f(m_run - m_new);
+                const float p0 = exp2f(z0 - m_new), p1 = exp2f(z1 - m_new);
+                float rs = p0 + p1;
+                rs += __shfl_xor_sync(0xffffffffu, rs, 1);
+                rs += __shfl_xor_sync(0xffffffffu, rs, 2);
+                l_run = l_run * corr + rs;
+                m_run = m_new;
+                // O^T columns are heads kc, kc + 1: fetch their corrections
+                const float ca = __shfl_sync(0xffffffffu, corr, 4 * kc);
+                const float cb = __shfl_sync(0xffffffffu, corr, 4 * kc + 4);
+    #pragma unroll
+                for (int i = 0; i < D / 16; ++i) { o[i][0] *= ca; o[i][1] *= cb; o[i][2] *= ca; o[i][3] *= cb; }
+                const uint32_t ph = pack_bf16x2(p0, p1);
+                const uint32_t pl = pack_bf16x2(p0 - bf16lo(ph), p1 - bf16hi(ph));
+                // O^T += V^T P^T; one ldmatrix.x4.trans covers two 16-dim row tiles
+    #pragma unroll
+                for (int m2 = 0; m2 < D / 32; ++m2) {
+                    uint32_t a[4];
+                    ldmatrix_x4_trans(a, st + (TB8 + mr) * RB + (((4 * m2 + mi) ^ mr) << 4));
+                    mma_bf16_1688(o[2 * m2], a[0], a[1], ph);
+                    mma_bf16_1688(o[2 * m2], a[0], a[1], pl);
+                    mma_bf16_1688(o[2 * m2 + 1], a[2], a[3], ph);
+                    mma_bf16_1688(o[2 * m2 + 1], a[2], a[3], pl);
+                }
+                __syncwarp();
+            }
+            cp_async_wait<0>();
             __syncwarp();
-            const uint8_t* st = ring + (bi % stages) * kStageBytes;
-            const int bt0 = (wid + bi * kNW) * TB8;
-            // Z = Q K^T over D in 16-dim steps; one ldmatrix.x4 covers 32 dims
-            float z[4] = {0.f, 0.f, 0.f, 0.f};
-            const int mr = lane & 7, mi = lane >> 3;  // ldmatrix: row (token) and matrix index
-#pragma unroll
-            for (int c4 = 0; c4 < D / 32; ++c4) {
-                uint32_t b[4];
-                ldmatrix_x4(b, st + mr * RB + (((4 * c4 + mi) ^ mr) << 4));
-                const uint2 q0 = qa[(2 * c4) * 32 + lane], q1 = qa[(2 * c4 + 1) * 32 + lane];
-                mma_bf16_16816(z, q0.x, 0u, q0.y, 0u, b[0], b[1]);
-                mma_bf16_16816(z, q1.x, 0u, q1.y, 0u, b[2], b[3]);
-            }
-            // online softmax for head hr over tokens kc, kc + 1 of the tile
-            const bool ok0 = bt0 + kc < n_att, ok1 = bt0 + kc + 1 < n_att;
-            const float z0 = ok0 ? z[0] * p.qscale : -INFINITY;
-            const float z1 = ok1 ? z[1] * p.qscale : -INFINITY;
-            float mx = fmaxf(z0, z1);
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            const float m_new = fmaxf(m_run, mx);
-            const float corr = exp2f(m_run - m_new);
-            const float p0 = exp2f(z0 - m_new), p1 = exp2f(z1 - m_new);
-            float rs = p0 + p1;
-            rs += __shfl_xor_sync(0xffffffffu, rs, 1);
-            rs += __shfl_xor_sync(0xffffffffu, rs, 2);
-            l_run = l_run * corr + rs;
-            m_run = m_new;
-            // O^T columns are heads kc, kc + 1: fetch their corrections
-            const float ca = __shfl_sync(0xffffffffu, corr, 4 * kc);
-            const float cb = __shfl_sync(0xffffffffu, corr, 4 * kc + 4);
-#pragma unroll
-            for (int i = 0; i < D / 16; ++i) { o[i][0] *= ca; o[i][1] *= cb; o[i][2] *= ca; o[i][3] *= cb; }
-            const uint32_t ph = pack_bf16x2(p0, p1);
-            const uint32_t pl = pack_bf16x2(p0 - bf16lo(ph), p1 - bf16hi(ph));
-            // O^T += V^T P^T; one ldmatrix.x4.trans covers two 16-dim row tiles
-#pragma unroll
-            for (int m2 = 0; m2 < D / 32; ++m2) {
-                uint32_t a[4];
-                ldmatrix_x4_trans(a, st + (TB8 + mr) * RB + (((4 * m2 + mi) ^ mr) << 4));
-                mma_bf16_1688(o[2 * m2], a[0], a[1], ph);
-                mma_bf16_1688(o[2 * m2], a[0], a[1], pl);
-                mma_bf16_1688(o[2 * m2 + 1], a[2], a[3], ph);
-                mma_bf16_1688(o[2 * m2 + 1], a[2], a[3], pl);
-            }
-            __syncwarp();
-        }
-        cp_async_wait<0>();
-        __syncwarp();
-        // [phase] 7
-        // per-warp partials -> the warp's own ring (its copies have all landed)
-        wp_out = reinterpret_cast<float*>(ring);
-#pragma unroll
-        for (int i = 0; i < D / 16; ++i) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int h = kc + (e & 1), d = 16 * i + hr + ((e & 2) ? 8 : 0);
-                if (h < G) wp_out[h * (D + 2) + d] = o[i][e];
-            }
-        }
-        if ((lane & 3) == 0 && hr < G) { wp_out[hr * (D + 2) + D] = m_run; wp_out[hr * (D + 2) + D + 1] = l_run; }
-    } else {
-        // fp32 K/V: CUDA cores. Each warp streams the K and V rows of its tokens
-        // through a ring of kAttStagesF32 shared-memory stages with cp.async
-        // (16-byte LDGSTS, no registers held while in flight), kAttStagesF32-1
-        // stages ahead of compute; lane l holds dims [l*EPL, l*EPL + EPL).
-        constexpr int kAttStages = kAttStagesF32;
-        constexpr int TBS = att_stage_tokens(RB, E::kBytes);      // tokens per stage
-        constexpr int kStageBytes = 2 * TBS * RB;
-        constexpr int kPiecesPerRow = RB / 16;
-        uint8_t* ring = smem + L.region + wid * att_ring_bytes(RB, E::kBytes, kAttStages);
-        const int nb = n_att > wid * TBS ? (n_att - wid * TBS + kNW * TBS - 1) / (kNW * TBS) : 0;
-        auto issue_stage = [&](int bi) {
-            const int bt0 = (wid + bi * kNW) * TBS;
-            uint8_t* st = ring + (bi % kAttStages) * kStageBytes;
-            for (int pc = lane; pc < 2 * TBS * kPiecesPerRow; pc += 32) {
-                const int r = pc / kPiecesPerRow, off = (pc - r * kPiecesPerRow) * 16;
-                const int u = r < TBS ? r : r - TBS;
-                if (bt0 + u < n_att) {
-                    const TKV* src = (r < TBS ? kb : vb) + (size_t)att_token(bt0 + u) * D;
-                    cp_async16(st + r * RB + off, reinterpret_cast<const uint8_t*>(src) + off);
+            // [phase] 7
+            // per-warp partials -> the warp's own ring (its copies have all landed)
+            wp_out = reinterpret_cast<float*>(ring);
+    #pragma unroll
+            for (int i = 0; i < D / 16; ++i) {
+    #pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int h = kc + (e & 1), d = 16 * i + hr + ((e & 2) ? 8 : 0);
+                    if (h < G) wp_out[h * (D + 2) + d] = o[i][e];
                 }
             }
-        };
-#pragma unroll 1
-        for (int bi = 0; bi < kAttStages - 1; ++bi) {
-            if (bi < nb) issue_stage(bi);
-            cp_async_commit();
-        }
-
-        float qf[GT][EPL];
-#pragma unroll
-        for (int h = 0; h < GT; ++h)
-#pragma unroll
-            for (int e = 0; e < EPL; ++e)
-                qf[h][e] = h < G ? qs[h * D + lane * EPL + e] * p.qscale : 0.f;
-
-        float m_run[GT], l_run[GT], o_run[GT][EPL];  // per query head of the group
-#pragma unroll
-        for (int h = 0; h < GT; ++h) {
-            m_run[h] = -INFINITY;
-            l_run[h] = 0.f;
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) o_run[h][e] = 0.f;
-        }
-
-        // [phase] 21
-#pragma unroll 1
-        for (int bi = 0; bi < nb; ++bi) {
-            if (bi + kAttStages - 1 < nb) issue_stage(bi + kAttStages - 1);
-            cp_async_commit();
-            cp_async_wait<kAttStages - 1>();
-            __syncwarp();
-            const uint8_t* st = ring + (bi % kAttStages) * kStageBytes;
-            const int bt0 = (wid + bi * kNW) * TBS;
-            bool ok[TBS];
-            float zt[TBS * GT];  // index u * GT + h
-#pragma unroll
-            for (int u = 0; u < TBS; ++u) {
-                ok[u] = bt0 + u < n_att;
-                uint32_t kw[RBL / 4 > 0 ? RBL / 4 : 1];
-                lds_words<RBL>(kw, st + u * RB + lane * RBL);
-                float kf[EPL];
-#pragma unroll
-                for (int e = 0; e < EPL; ++e) {
-                    if constexpr (E::kBytes == 2) kf[e] = (e & 1) ? bf16hi(kw[e >> 1]) : bf16lo(kw[e >> 1]);
-                    else kf[e] = __uint_as_float(kw[e]);
-                }
-#pragma unroll
-                for (int h = 0; h < GT; ++h) {
-                    float a = 0.f;
-#pragma unroll
-                    for (int e = 0; e < EPL; ++e) a = fmaf(qf[h][e], kf[e], a);
-                    zt[u * GT + h] = a;
-                }
-            }
-            warp_allreduce_n<TBS * GT>(zt);
-#pragma unroll
-            for (int h = 0; h < GT; ++h) {
-                if (h >= G) break;
-                float mx = -INFINITY;
-#pragma unroll
-                for (int u = 0; u < TBS; ++u) if (ok[u]) mx = fmaxf(mx, zt[u * GT + h]);
-                const float m_new = fmaxf(m_run[h], mx);
-                const float corr = exp2f(m_run[h] - m_new);
-                float l = l_run[h] * corr;
-#pragma unroll
-                for (int e = 0; e < EPL; ++e) o_run[h][e] *= corr;
-#pragma unroll
-                for (int u = 0; u < TBS; ++u) {
-                    if (!ok[u]) continue;
-                    const float pr = exp2f(zt[u * GT + h] - m_new);
-                    l += pr;
-                    uint32_t vw[RBL / 4 > 0 ? RBL / 4 : 1];
-                    lds_words<RBL>(vw, st + (TBS + u) * RB + lane * RBL);
-#pragma unroll
-                    for (int e = 0; e < EPL; ++e) {
-                        float vf;
-                        if constexpr (E::kBytes == 2) vf = (e & 1) ? bf16hi(vw[e >> 1]) : bf16lo(vw[e >> 1]);
-                        else vf = __uint_as_float(vw[e]);
-                        o_run[h][e] = fmaf(pr, vf, o_run[h][e]);
+            if ((lane & 3) == 0 && hr < G) { wp_out[hr * (D + 2) + D] = m_run; wp_out[hr * (D + 2) + D + 1] = l_run; }
+        } else {
+            // fp32 K/V: CUDA cores. Each warp streams the K and V rows of its tokens
+            // through a ring of kAttStagesF32 shared-memory stages with cp.async
+            // (16-byte LDGSTS, no registers held while in flight), kAttStagesF32-1
+            // stages ahead of compute; lane l holds dims [l*EPL, l*EPL + EPL).
+            constexpr int kAttStages = kAttStagesF32;
+            constexpr int TBS = att_stage_tokens(RB, E::kBytes);      // tokens per stage
+            constexpr int kStageBytes = 2 * TBS * RB;
+            constexpr int kPiecesPerRow = RB / 16;
+            uint8_t* ring = smem + L.region + wid * att_ring_bytes(RB, E::kBytes, kAttStages);
+            const int nb = n_att > wid * TBS ? (n_att - wid * TBS + kNW * TBS - 1) / (kNW * TBS) : 0;
+            auto issue_stage = [&](int bi) {
+                const int bt0 = (wid + bi * kNW) * TBS;
+                uint8_t* st = ring + (bi % kAttStages) * kStageBytes;
+                for (int pc = lane; pc < 2 * TBS * kPiecesPerRow; pc += 32) {
+                    const int r = pc / kPiecesPerRow, off = (pc - r * kPiecesPerRow) * 16;
+                    const int u = r < TBS ? r : r - TBS;
+                    if (bt0 + u < n_att) {
+                        const TKV* src = (r < TBS ? kb : vb) + att_row(bt0 + u) * D;
+                        cp_async16(st + r * RB + off, reinterpret_cast<const uint8_t*>(src) + off);
                     }
                 }
-                m_run[h] = m_new;
-                l_run[h] = l;
+            };
+    #pragma unroll 1
+            for (int bi = 0; bi < kAttStages - 1; ++bi) {
+                if (bi < nb) issue_stage(bi);
+                cp_async_commit();
             }
-            __syncwarp();
-        }
-        cp_async_wait<0>();
-        __syncwarp();
 
-        // [phase] 7
-        // per-warp partials -> the warp's own ring (its copies have all landed)
-        wp_out = reinterpret_cast<float*>(ring);
-        {
-        float* wp = wp_out;
-#pragma unroll
-        for (int h = 0; h < GT; ++h) {
-            if (h >= G) break;
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) wp[h * (D + 2) + lane * EPL + e] = o_run[h][e];
-            if (lane == 0) { wp[h * (D + 2) + D] = m_run[h]; wp[h * (D + 2) + D + 1] = l_run[h]; }
+            float qf[GT][EPL];
+    #pragma unroll
+            for (int h = 0; h < GT; ++h)
+    #pragma unroll
+                for (int e = 0; e < EPL; ++e)
+                    qf[h][e] = h < G ? qs[h * D + lane * EPL + e] * p.qscale : 0.f;
+
+            float m_run[GT], l_run[GT], o_run[GT][EPL];  // per query head of the group
+    #pragma unroll
+            for (int h = 0; h < GT; ++h) {
+                m_run[h] = -INFINITY;
+                l_run[h] = 0.f;
+    #pragma unroll
+                for (int e = 0; e < EPL; ++e) o_run[h][e] = 0.f;
+            }
+
+            // [phase] 21
+    #pragma unroll 1
+            for (int bi = 0; bi < nb; ++bi) {
+                if (bi + kAttStages - 1 < nb) issue_stage(bi + kAttStages - 1);
+                cp_async_commit();
+                cp_async_wait<kAttStages - 1>();
+                __syncwarp();
+                const uint8_t* st = ring + (bi % kAttStages) * kStageBytes;
+                const int bt0 = (wid + bi * kNW) * TBS;
+                bool ok[TBS];
+                float zt[TBS * GT];  // index u * GT + h
+    #pragma unroll
+                for (int u = 0; u < TBS; ++u) {
+                    ok[u] = bt0 + u < n_att;
+                    uint32_t kw[RBL / 4 > 0 ? RBL / 4 : 1];
+                    lds_words<RBL>(kw, st + u * RB + lane * RBL);
+                    float kf[EPL];
+    #pragma unroll
+                    for (int e = 0; e < EPL; ++e) {
+                        if constexpr (E::kBytes == 2) kf[e] = (e & 1) ? bf16hi(kw[e >> 1]) : bf16lo(kw[e >> 1]);
+                        else kf[e] = __uint_as_float(kw[e]);
+                    }
+    #pragma unroll
+                    for (int h = 0; h < GT; ++h) {
+                        float a = 0.f;
+    #pragma unroll
+                        for (int e = 0; e < EPL; ++e) a = fmaf(qf[h][e], kf[e], a);
+                        zt[u * GT + h] = a;
+                    }
+                }
+                warp_allreduce_n<TBS * GT>(zt);
+    #pragma unroll
+                for (int h = 0; h < GT; ++h) {
+                    if (h >= G) break;
+                    float mx = -INFINITY;
+    #pragma unroll
+                    for (int u = 0; u < TBS; ++u) if (ok[u]) mx = fmaxf(mx, zt[u * GT + h]);
+                    const float m_new = fmaxf(m_run[h], mx);
+                    const float corr = exp2f(m_run[h] - m_new);
+                    float l = l_run[h] * corr;
+    #pragma unroll
+                    for (int e = 0; e < EPL; ++e) o_run[h][e] *= corr;
+    #pragma unroll
+                    for (int u = 0; u < TBS; ++u) {
+                        if (!ok[u]) continue;
+                        const float pr = exp2f(zt[u * GT + h] - m_new);
+                        l += pr;
+                        uint32_t vw[RBL / 4 > 0 ? RBL / 4 : 1];
+                        lds_words<RBL>(vw, st + (TBS + u) * RB + lane * RBL);
+    #pragma unroll
+                        for (int e = 0; e < EPL; ++e) {
+                            float vf;
+                            if constexpr (E::kBytes == 2) vf = (e & 1) ? bf16hi(vw[e >> 1]) : bf16lo(vw[e >> 1]);
+                            else vf = __uint_as_float(vw[e]);
+                            o_run[h][e] = fmaf(pr, vf, o_run[h][e]);
+                        }
+                    }
+                    m_run[h] = m_new;
+                    l_run[h] = l;
+                }
+                __syncwarp();
+            }
+            cp_async_wait<0>();
+            __syncwarp();
+
+            // [phase] 7
+            // per-warp partials -> the warp's own ring (its copies have all landed)
+            wp_out = reinterpret_cast<float*>(ring);
+            {
+            float* wp = wp_out;
+    #pragma unroll
+            for (int h = 0; h < GT; ++h) {
+                if (h >= G) break;
+    #pragma unroll
+                for (int e = 0; e < EPL; ++e) wp[h * (D + 2) + lane * EPL + e] = o_run[h][e];
+                if (lane == 0) { wp[h * (D + 2) + D] = m_run[h]; wp[h * (D + 2) + D + 1] = l_run[h]; }
+            }
         }
-    }
-    }
+        }
+    };
+    if (p.block_table)
+        attend([&](int j) -> size_t {
+            return select_all ? kv_row_of(p, row / p.hkv, g, row_tok, t0 + j) : (size_t)sel_rows[j];
+        });
+    else
+        attend([&](int j) -> size_t { return row_tok + (size_t)(select_all ? t0 + j : sel_list[j]); });
     __syncthreads();
     // merge the warps' states per head; a single-CTA row writes its output here
     for (int e = tid; e < G * D; e += kNT) {

@@ -25,6 +25,8 @@ struct LabelArgs {
     void* label;
     uint16_t* lscale;
     uint16_t* lzero;
+    const int32_t* block_table = nullptr;  // paged key cache (see ds_label.cu)
+    int max_blocks = 0, page_shift = 0, num_blocks = 0;
 };
 cudaError_t launch_label(const LabelArgs& a, cudaStream_t st);
 

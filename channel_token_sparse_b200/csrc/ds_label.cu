@@ -8,6 +8,9 @@
 // One CTA handles kTokens consecutive tokens of one (b, kv head) row: the key
 // rows are staged in shared memory with coalesced 16-byte loads, then each
 // label element (fp) or each token (4-bit) is produced from shared memory.
+// The key cache is dense [b, hkv, s_cap, d] or paged (a block table maps
+// token t of entry b to a row of a [num_blocks, hkv, page, d] pool); the
+// label cache is always dense [b, hkv, s_cap, c].
 #include "ds_common.cuh"
 #include "ds_internal.h"
 
@@ -22,7 +25,9 @@ __global__ void __launch_bounds__(kLabNT) ds_label_kernel(const TKV* __restrict_
                                                           int t_begin, int t_end, int s_cap, int c,
                                                           uint8_t* __restrict__ label,
                                                           uint16_t* __restrict__ lscale,
-                                                          uint16_t* __restrict__ lzero) {
+                                                          uint16_t* __restrict__ lzero,
+                                                          const int32_t* __restrict__ block_table,
+                                                          int max_blocks, int page_shift, int num_blocks) {
     using E = Elem<TKV>;
     __shared__ __align__(16) TKV rows[kTokens * D];
     __shared__ int idx_s[128];
@@ -35,9 +40,20 @@ __global__ void __launch_bounds__(kLabNT) ds_label_kernel(const TKV* __restrict_
 
     const size_t tok0 = (size_t)row * s_cap + tb;
     constexpr int kVecPerRow = D * E::kBytes / 16;
-    const uint4* src = reinterpret_cast<const uint4*>(k + tok0 * D);
     uint4* dst = reinterpret_cast<uint4*>(rows);
-    for (int e = threadIdx.x; e < nt * kVecPerRow; e += kLabNT) dst[e] = ldg_stream16(src + e);
+    if (!block_table) {
+        const uint4* src = reinterpret_cast<const uint4*>(k + tok0 * D);
+        for (int e = threadIdx.x; e < nt * kVecPerRow; e += kLabNT) dst[e] = ldg_stream16(src + e);
+    } else {
+        const int32_t* bt = block_table + (size_t)(row / hkv) * max_blocks;
+        const int pmask = (1 << page_shift) - 1;
+        for (int e = threadIdx.x; e < nt * kVecPerRow; e += kLabNT) {
+            const int t = tb + e / kVecPerRow;
+            const int blk = min(max(__ldg(bt + (t >> page_shift)), 0), num_blocks - 1);
+            const size_t r = (((size_t)blk * hkv + g) << page_shift) + (size_t)(t & pmask);
+            dst[e] = ldg_stream16(reinterpret_cast<const uint4*>(k + r * D) + e % kVecPerRow);
+        }
+    }
     __syncthreads();
 
     if constexpr (LK == 0) {
@@ -60,7 +76,8 @@ static cudaError_t launch_label_t(const LabelArgs& a, cudaStream_t st) {
     dim3 grid((n + kTokens - 1) / kTokens, a.b * a.hkv);
     ds_label_kernel<TKV, LK, D><<<grid, kLabNT, 0, st>>>(
         reinterpret_cast<const TKV*>(a.k), a.idx, a.hkv, a.t_begin, a.t_end, a.s_cap, a.c,
-        reinterpret_cast<uint8_t*>(a.label), a.lscale, a.lzero);
+        reinterpret_cast<uint8_t*>(a.label), a.lscale, a.lzero, a.block_table, a.max_blocks, a.page_shift,
+        a.num_blocks);
     return cudaGetLastError();
 }
 

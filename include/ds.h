@@ -245,6 +245,39 @@ DS_API ds_status ds_decode_step_varlen(const void* q, const void* k, const void*
                                        int topk, float sm_scale, void* out, ds_dtype out_dt,
                                        int32_t* sel_out, float* score_out, cudaStream_t stream);
 
+/* ------------------------------------------------------------ paged K/V
+ * The serving layout the pages' SGLang section implies (a shared pool of
+ * fixed-size pages instead of one contiguous cache per sequence). The key and
+ * value pools are [num_blocks, hkv, page_size, d] (dtype kdt / kvdt) and
+ * block_table [b, max_blocks] (int32, device) names, for batch entry b, the
+ * block that holds its tokens [j * page_size, (j + 1) * page_size): token t
+ * is row t % page_size of block block_table[b * max_blocks + t / page_size].
+ * Block ids are clamped into [0, num_blocks). page_size is a power of two in
+ * [1, 65536], max_blocks * page_size >= the token count, and
+ * num_blocks * hkv * page_size < 2^32. The label cache stays dense
+ * [b, hkv, s_cap, c] (s_cap is its capacity). block_table needs 4-byte
+ * alignment, the pools 16. Same results as the dense-layout calls on the
+ * same values. */
+
+/* ds_build_label_cache for a paged key pool: label rows [0, s). */
+DS_API ds_status ds_build_label_cache_paged(const void* k_pool, ds_dtype kdt, const int32_t* idx,
+                                            const int32_t* block_table, int max_blocks,
+                                            int page_size, int num_blocks, int b, int hkv, int s,
+                                            int s_cap, int d, int c, void* label, ds_dtype label_dt,
+                                            uint16_t* lscale, uint16_t* lzero, cudaStream_t stream);
+
+/* ds_decode_step_varlen over paged K/V pools. seq_lens may be NULL (every
+ * entry has s_max tokens). */
+DS_API ds_status ds_decode_step_paged(const void* q, const void* k_pool, const void* v_pool,
+                                      ds_dtype kvdt, void* label, ds_dtype label_dt,
+                                      uint16_t* lscale, uint16_t* lzero, const int32_t* idx,
+                                      const int32_t* block_table, int max_blocks, int page_size,
+                                      int num_blocks, const int32_t* seq_lens,
+                                      int sparse_threshold, ds_fallback fallback,
+                                      int b, int hq, int hkv, int s_max, int s_cap, int d, int c,
+                                      int topk, float sm_scale, void* out, ds_dtype out_dt,
+                                      int32_t* sel_out, float* score_out, cudaStream_t stream);
+
 /* Launch plan of ds_sparse_decode for a shape (host only, launches nothing):
  * CTAs per thread-block cluster (one cluster per (b, kv head)), tokens per
  * CTA and dynamic shared memory per CTA in bytes. Any output may be NULL. */

@@ -6,6 +6,8 @@ within 1e-4 relative of the k-th score; outputs within max-abs 2e-3 of the
 oracle's attention over the GPU's selected set.
 """
 
+import dataclasses
+
 import numpy as np
 import pytest
 
@@ -274,8 +276,10 @@ def test_calibration_matches_oracle_and_recovers_outliers(wl_i):
 
 # ------------------------------------------------------ full-size configs
 
-def _full_config(i, rows_to_check):
+def _full_config(i, rows_to_check, label_dtype=None):
     wl = synth.workload(i)
+    if label_dtype:
+        wl = dataclasses.replace(wl, label_dtype=label_dtype)
     if i == 0:
         # heavy channels from calibration on the 4 samples (= the planted set, pinned on CPU)
         run_decode_case(wl, idx=synth.outlier_channels(wl))
@@ -341,6 +345,17 @@ def _full_config(i, rows_to_check):
 ])
 def test_full_size_configs(i, rows):
     _full_config(i, rows)
+
+
+@pytest.mark.parametrize("i,rows", [
+    (1, [(0, 0), (5, 9)]),
+    (3, [(1, 2)]),
+    (4, [(0, 5)]),
+])
+def test_int4_labels_at_bf16_label_shapes(i, rows):
+    """The 4-bit label cache (16 channels: 8 payload bytes + fp16 scale and
+    zero per token) on the Llama-2-7B, GQA and 256K shapes."""
+    _full_config(i, rows, label_dtype="int4")
 
 
 # ------------------------------------------------------- fused decode step

@@ -6,6 +6,7 @@
   short entries (per entry, or for the whole batch as SGLang states it);
 - key/value caches in pinned host memory read by the kernels over the host
   link (Double Sparsity's offloading mode), bit-identical to device caches;
+- paged K/V pools with a block table, bit-identical to the dense layout;
 - the channel criteria of ds_calibrate_channels_criterion (Q-, K-, QK-outlier,
   chunked QK norm, LeanK ratio): channel indices bit-exact.
 """
@@ -315,3 +316,86 @@ def test_criteria_reject_bad_arguments():
         ds.calibrate_channels_criterion(q, k, 8, ds.DS_CRIT_QK_CHUNKED, 0)
     with pytest.raises(ds.DSError):
         ds.calibrate_channels_criterion(q, k, 8, 7)
+
+
+# --------------------------------------------------------------- paged K/V
+
+def _to_pool(x, page, seed):
+    """Scatter a dense cache [B, Hkv, S_cap, D] into a pool [num_blocks, Hkv,
+    page, D] of shuffled blocks (plus unused ones); returns (pool, table)."""
+    b, hkv, s_cap, d = x.shape
+    mb = (s_cap + page - 1) // page
+    nblk = b * mb + 5
+    perm = torch.from_numpy(np.random.default_rng(seed).permutation(nblk)[: b * mb].astype(np.int32))
+    table = perm.view(b, mb).cuda()
+    pool = torch.zeros((nblk, hkv, page, d), dtype=x.dtype, device=x.device)
+    pad = torch.zeros((b, hkv, mb * page, d), dtype=x.dtype, device=x.device)
+    pad[:, :, :s_cap] = x
+    blocks = pad.view(b, hkv, mb, page, d).permute(0, 2, 1, 3, 4).reshape(b * mb, hkv, page, d)
+    pool[perm.long().cuda()] = blocks
+    return pool, table
+
+
+@pytest.mark.parametrize("kv,label,page,varlen,cluster", [
+    ("bf16", "bf16", 16, False, 0), ("bf16", "int4", 64, True, 0), ("f32", "f32", 8, True, 2),
+    ("bf16", "bf16", 1, False, 4), ("bf16", "bf16", 256, True, 1)])
+def test_paged_kv_equals_dense_layout(kv, label, page, varlen, cluster):
+    """The paged pools give the same bits as the dense caches holding the
+    same values: label build, decode step (per-entry lengths too)."""
+    b, hq, hkv, d, c, s, topk = 3, 8, 4, 128, 16 if label != "int4" else 32, 3000, 256
+    if kv == "f32":
+        d, c = 64, 8
+    wl = synth.custom(b=b, hq=hq, hkv=hkv, d=d, s=s, c=c, topk=topk, kv_dtype=kv, label_dtype=label,
+                      n_outlier=min(16, c), outlier_scale=6.0, index=85)
+    di = synth.decode_inputs(wl, s_cap=s + 8)
+    idx = _idx_random(wl, 13)
+    qd, kd, vd = (to_dev(x, kv) for x in (di.q, di.k, di.v))
+    idxd = torch.from_numpy(idx).cuda()
+    kp, table = _to_pool(kd, page, 5)
+    vp, table_v = _to_pool(vd, page, 5)
+    assert torch.equal(table, table_v)
+    lab1, sc1, ze1 = _label_alloc(kd, wl)
+    lab2, sc2, ze2 = _label_alloc(kd, wl)
+    ds.build_label_cache(kd, idxd, s - 1, lab1, sc1, ze1)
+    ds.build_label_cache_paged(kp, idxd, table, s - 1, lab2, sc2, ze2)
+    torch.cuda.synchronize()
+    assert torch.equal(lab1, lab2)
+    if sc1 is not None:
+        assert torch.equal(sc1, sc2) and torch.equal(ze1, ze2)
+    lens = torch.tensor([s, 1700, 200][:b], dtype=torch.int32, device="cuda") if varlen else None
+    sel1 = torch.full((b, hkv, topk), -7, dtype=torch.int32, device="cuda")
+    sel2 = sel1.clone()
+    ds.set_cluster(cluster)
+    try:
+        if varlen:
+            o1 = ds.decode_step_varlen(qd, kd, vd, lab1, idxd, lens, s, topk, lscale=sc1, lzero=ze1, sel_out=sel1)
+        else:
+            o1 = ds.decode_step(qd, kd, vd, lab1, idxd, s, topk, lscale=sc1, lzero=ze1, sel_out=sel1)
+        o2 = ds.decode_step_paged(qd, kp, vp, lab2, idxd, table, s, topk, seq_lens=lens, lscale=sc2, lzero=ze2,
+                                  sel_out=sel2)
+        torch.cuda.synchronize()
+    finally:
+        ds.set_cluster(0)
+    assert torch.equal(lab1, lab2) and torch.equal(sel1, sel2) and torch.equal(o1, o2)
+    if not varlen:      # and the oracle agrees
+        ref_label = oracle.build_label(di.k, kv, label, idx, s)
+        _, sel_ref, s_ref = oracle.sparse_decode(di.q, di.k, di.v, kv, ref_label, label, idx, s, topk)
+        sg = sel2.cpu().numpy()
+        check_selection(sg.reshape(-1, topk), sel_ref.reshape(-1, topk), s_ref.reshape(-1, s), topk, s)
+        o_ref = oracle.attention(di.q, di.k, di.v, kv, sg, hkv)
+        assert np.abs(o2.cpu().numpy() - o_ref).max() <= OUT_ATOL
+
+
+def test_paged_rejects_bad_tables():
+    q = torch.zeros((1, 2, 64), device="cuda")
+    pool = torch.zeros((4, 2, 16, 64), device="cuda")
+    lab = torch.zeros((1, 2, 64, 8), device="cuda")
+    idx = torch.zeros((2, 8), dtype=torch.int32, device="cuda")
+    table = torch.zeros((1, 4), dtype=torch.int32, device="cuda")
+    with pytest.raises(ds.DSError):      # 4 blocks of 16 cannot hold 65 tokens
+        ds.decode_step_paged(q, pool, pool, torch.zeros((1, 2, 80, 8), device="cuda"), idx, table, 65, 16)
+    with pytest.raises(ds.DSError):      # page size not a power of two
+        ds.decode_step_paged(q, torch.zeros((4, 2, 12, 64), device="cuda"), torch.zeros((4, 2, 12, 64), device="cuda"),
+                             lab, idx, table, 40, 16)
+    ds.decode_step_paged(q, pool, pool, lab, idx, table, 64, 16)   # valid
+    torch.cuda.synchronize()
