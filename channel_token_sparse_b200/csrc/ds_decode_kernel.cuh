@@ -530,14 +530,16 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
                 if (grp >= wg1) continue;
                 uint32_t w[4];
                 key8(grp, w);
-                uint32_t flags = 0;
+                uint32_t flags = 0, above = 0;
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const bool ok = grp * 8 + e < n_loc;
                     if (ok && kat(w, e) == T16) flags |= 1u << e;
-                    above_cnt += ok && kat(w, e) > T16;
+                    if (ok && kat(w, e) > T16) above |= 1u << e;
                 }
+                above_cnt += __popc(above);
                 bits8[grp] = (uint8_t)flags;
+                mcache[grp] = (uint16_t)above;   // keys selected outright, for the write pass
                 for (uint32_t m = flags; m; m &= m - 1) {
                     const int i = grp * 8 + __ffs(m) - 1;
                     const uint32_t low = p.keep_low ? (uint32_t)low16[i] : score_key(rescore(i)) & 0xFFFFu;
@@ -637,6 +639,23 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         // bucket tokens; otherwise a count pass classifies every key (and
         // keeps each group's masks, 2 bytes, for the write pass).
         const bool counts_known = refine && ctl[kCtlBL] <= kBucketCap;
+        // With the counts known, a group's masks are the refine sweep's
+        // "above" bits plus its bucket tokens classified by their low bits.
+        auto masks_swept = [&](int grp) -> uint32_t {
+            uint32_t m = mcache[grp];
+            const uint32_t fl = bits8[grp];
+            if (fl) {
+                uint32_t w[4];
+                key8(grp, w);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if ((fl >> e) & 1u) {
+                        const int low = kat(w, e);
+                        m |= low > Tlo ? (1u << e) : (low == Tlo ? (1u << (8 + e)) : 0u);
+                    }
+            }
+            return m;
+        };
         if (counts_known) {
             const int nbl = ctl[kCtlBL];
             for (int j = tid; j < nbl; j += kNT) {
@@ -698,7 +717,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         int cur_dst = -1;
         int* rl = nullptr;
         for (int grp = wg0 + lane; grp - lane < wg1; grp += 32) {
-            const uint32_t m = grp < wg1 ? (counts_known ? masks8(grp) : (uint32_t)mcache[grp]) : 0u;
+            const uint32_t m = grp < wg1 ? (counts_known ? masks_swept(grp) : (uint32_t)mcache[grp]) : 0u;
             const uint32_t smk = m & 255u, tmk = m >> 8;
             const uint32_t pk = ((uint32_t)__popc(smk) << 16) | (uint32_t)__popc(tmk);
             const uint32_t incl = warp_incl_scan(pk);
@@ -713,11 +732,15 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
                 const int t_before = my_tb + __popc(tmk & below);
                 if (((tmk >> e) & 1u) && t_before >= tie_quota) continue;  // tie beyond the quota
                 const uint32_t pos = (uint32_t)(P + s_before + min(t_before, tie_quota));
-                uint32_t dst = __umulhi(pos, per_inv);
-                if ((dst + 1u) * per <= pos) ++dst;
-                if ((int)dst != cur_dst) { cur_dst = (int)dst; rl = row_smem(cluster, N, sel_list, (int)dst); }
                 const int t = t0 + grp * 8 + e;
-                rl[pos - dst * per] = t;
+                if (N == 1) {
+                    sel_list[pos] = t;
+                } else {
+                    uint32_t dst = __umulhi(pos, per_inv);
+                    if ((dst + 1u) * per <= pos) ++dst;
+                    if ((int)dst != cur_dst) { cur_dst = (int)dst; rl = row_smem(cluster, N, sel_list, (int)dst); }
+                    rl[pos - dst * per] = t;
+                }
                 if (p.sel_out) p.sel_out[(size_t)row * p.topk + pos] = t;
             }
         }
