@@ -34,6 +34,8 @@ SIGNATURES = {
     "ds_calibrate_workspace_size": (_i, [_i, _i, _i, _i, _i, _i, C.POINTER(_sz)]),
     "ds_calibrate_channels": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp]),
     "ds_calibrate_channels_noalloc": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "ds_decode_step_kv": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                               _i, _f, _vp, _i, _vp, _vp, _vp]),
     "ds_build_label_cache_paged": (_i, [_vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _i, _vp,
                                         _vp, _vp]),
     "ds_decode_step_paged": (_i, [_vp, _vp, _vp, _i, _vp, _i, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _i, _i, _i,
@@ -309,6 +311,30 @@ def decode_step(q, k, v, label, idx, s: int, topk: int, lscale=None, lzero=None,
                                 _label_args(label, lscale, lzero, kdt), _ptr(lscale), _ptr(lzero),
                                 _ptr(idx), b, hq, hkv, s, s_cap, d, c, topk, float(sm_scale),
                                 _ptr(out), odt, _ptr(sel_out), _ptr(score_out), _stream(stream)))
+    return out
+
+
+def decode_step_kv(q, k_new, v_new, k, v, label, idx, s: int, topk: int, lscale=None, lzero=None, out=None,
+                   out_dtype=None, sm_scale: float = 0.0, sel_out=None, score_out=None, stream=None):
+    """decode_step that first writes the new token's rows k_new, v_new
+    [B, Hkv, D] into k, v at position s - 1 (in the same launch); returns
+    out [B, Hq, D]."""
+    torch = _torch()
+    _need_cuda_or_pinned(k, v)
+    _need_cuda(q, k_new, v_new, label, idx, lscale, lzero, out, sel_out, score_out)
+    b, hq, d = q.shape
+    _, hkv, s_cap, _ = k.shape
+    c = idx.shape[1]
+    kdt = _kv_dtype(k)
+    if k_new.dtype != k.dtype or v_new.dtype != v.dtype:
+        raise TypeError("k_new / v_new must have the caches' dtype")
+    if out is None:
+        out = torch.empty((b, hq, d), dtype=out_dtype or torch.float32, device=q.device)
+    odt = DS_F32 if out.dtype == torch.float32 else DS_BF16
+    _check(lib().ds_decode_step_kv(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr_kv(k), _ptr_kv(v), kdt, _ptr(label),
+                                   _label_args(label, lscale, lzero, kdt), _ptr(lscale), _ptr(lzero),
+                                   _ptr(idx), b, hq, hkv, s, s_cap, d, c, topk, float(sm_scale),
+                                   _ptr(out), odt, _ptr(sel_out), _ptr(score_out), _stream(stream)))
     return out
 
 

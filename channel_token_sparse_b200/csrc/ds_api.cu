@@ -388,10 +388,13 @@ ds_status sparse_decode_impl(const void* q, const void* k, const void* v, ds_dty
                              const int32_t* idx, int b, int hq, int hkv, int s, int s_cap, int d, int c,
                              int topk, float sm_scale, void* out, ds_dtype out_dt, int32_t* sel_out,
                              float* score_out, bool append, const int32_t* seq_lens, int threshold,
-                             int batch_rule, cudaStream_t stream, const Paged* pg = nullptr) {
+                             int batch_rule, cudaStream_t stream, const Paged* pg = nullptr,
+                             const void* k_new = nullptr, const void* v_new = nullptr) {
     ds_status r = check_common(b, hq, hkv, s, s_cap, d, kvdt);
     if (r != DS_OK) return r;
     if (pg && (r = check_paged(*pg, s, hkv, d)) != DS_OK) return r;
+    if ((k_new == nullptr) != (v_new == nullptr)) return fail(DS_ERR_INVALID_ARG, "give both k_new and v_new or neither");
+    if (k_new && (!aligned16(k_new) || !aligned16(v_new))) return fail(DS_ERR_INVALID_ARG, "k_new/v_new not 16-byte aligned");
     if ((r = check_label(kvdt, label_dt, c, d, label, lscale, lzero)) != DS_OK) return r;
     if (topk < 1) return fail(DS_ERR_INVALID_ARG, "topk must be >= 1");
     if (!q || !k || !v || !idx || !out) return fail(DS_ERR_INVALID_ARG, "NULL pointer");
@@ -417,6 +420,8 @@ ds_status sparse_decode_impl(const void* q, const void* k, const void* v, ds_dty
     p.nb = b;
     p.threshold = threshold;
     p.batch_rule = batch_rule;
+    p.k_new = k_new;
+    p.v_new = v_new;
     if (pg) {
         p.block_table = pg->bt;
         p.max_blocks = pg->max_blocks;
@@ -457,6 +462,16 @@ ds_status ds_decode_step(const void* q, const void* k, const void* v, ds_dtype k
                          cudaStream_t stream) {
     return sparse_decode_impl(q, k, v, kvdt, label, label_dt, lscale, lzero, idx, b, hq, hkv, s, s_cap, d, c,
                               topk, sm_scale, out, out_dt, sel_out, score_out, true, nullptr, 0, 0, stream);
+}
+
+ds_status ds_decode_step_kv(const void* q, const void* k_new, const void* v_new, void* k, void* v, ds_dtype kvdt,
+                            void* label, ds_dtype label_dt, uint16_t* lscale, uint16_t* lzero, const int32_t* idx,
+                            int b, int hq, int hkv, int s, int s_cap, int d, int c, int topk, float sm_scale,
+                            void* out, ds_dtype out_dt, int32_t* sel_out, float* score_out, cudaStream_t stream) {
+    if (!k_new || !v_new) return fail(DS_ERR_INVALID_ARG, "k_new or v_new is NULL");
+    return sparse_decode_impl(q, k, v, kvdt, label, label_dt, lscale, lzero, idx, b, hq, hkv, s, s_cap, d, c,
+                              topk, sm_scale, out, out_dt, sel_out, score_out, true, nullptr, 0, 0, stream, nullptr,
+                              k_new, v_new);
 }
 
 ds_status ds_decode_step_varlen(const void* q, const void* k, const void* v, ds_dtype kvdt, void* label,

@@ -71,6 +71,10 @@ struct DecodeParams {
     // row t & (page - 1) of block block_table[b * max_blocks + (t >> page_shift)]
     const int32_t* block_table;
     int max_blocks, page_shift, num_blocks;
+    // decode step with the new token's rows given ([b, hkv, d] each, or null):
+    // the kernel writes them into the K/V caches at position s-1 itself
+    const void* k_new;
+    const void* v_new;
 };
 
 // Row (in units of d elements) of token t of (b, g) in the K/V caches, dense
@@ -108,6 +112,7 @@ __host__ __device__ constexpr int att_ring_bytes(int row_bytes, int elem_bytes, 
 // Tokens of the k-th key's 16-bit bucket kept in a list for the last radix
 // pass (a CTA whose bucket is larger falls back to sweeping its keys).
 constexpr int kBucketCap = 1024;
+constexpr int kMaxCluster = 16;  // CTAs per row at most (portable 8, non-portable 16)
 
 __host__ __device__ inline DecodeSmem decode_smem_layout(int GT, int D, int C, int chunk, int per,
                                                          int elem_bytes, int att_stages) {
@@ -121,9 +126,9 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int GT, int D, int C, i
     L.histB = o;  o += 256 * 4;
     L.ctl = o;    o += 64 * 4;
     L.scan = o;   o += align16((kNW + 1) * 4);
-    L.cm = o;     o += align16(GT * 4);
-    L.cl = o;     o += align16(GT * 4);
-    L.co = o;     o += align16(GT * D * 4);
+    L.cm = o;     o += align16(kMaxCluster * GT * 4);        // cluster merge: (m, l) of every CTA
+    L.cl = o;     o += align16(kMaxCluster * GT * 4);
+    L.co = o;     o += align16((GT * D + kMaxCluster) * 4);  // cluster merge: partial o received
     L.bits = o;   o += align16(chunk / 8);
     L.mcache = o; o += align16(chunk / 8 * 2);  // per key group: selected / tie masks
     L.blist = o;  o += chunk > 0 ? kBucketCap * 4 : 0;
@@ -139,7 +144,8 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int GT, int D, int C, i
 
 // ctl[] slots
 enum { kCtlBin = 0, kCtlNeed = 1, kCtlCnt = 2, kCtlCS = 4, kCtlCT = 5, kCtlP = 6, kCtlTP = 7, kCtlBL = 8,
-       kCtlTlo = 9, kCtlTie = 10, kCtlWarp = 16 /* kNW per-warp packed counts */ };
+       kCtlTlo = 9, kCtlTie = 10, kCtlWarp = 16 /* kNW per-warp packed counts */,
+       kCtlGather = 32 /* 16 per-CTA bucket-list offsets, then the total */ };
 
 // Row geometry of the label cache.
 template <typename TKV, int LK, int C>
@@ -214,8 +220,14 @@ __device__ __forceinline__ void cluster_select_bin(cg::cluster_group& cluster, u
     uint32_t cnt = 0;
     for (int r = 0; r < nblocks; ++r) cnt += row_smem(cluster, nblocks, hist, r)[bin];
     if (zero_next) zero_next[tid] = 0u;
-    uint32_t total;
-    const uint32_t excl = block_excl_scan<kNT>(cnt, scan, &total);
+    // prefix over bins (largest first): warp scans, then every warp adds the
+    // totals of the warps before it (one barrier, no second scan)
+    const uint32_t incl = warp_incl_scan(cnt);
+    if (lane_id() == 31) scan[warp_id()] = incl;
+    __syncthreads();
+    uint32_t excl = incl - cnt;
+#pragma unroll
+    for (int w = 0; w < kNW; ++w) excl += w < warp_id() ? scan[w] : 0u;
     if (excl < need && need <= excl + cnt) {
         ctl[kCtlBin] = bin;
         ctl[kCtlNeed] = (int)(need - excl);
@@ -307,10 +319,16 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     }
     const int iv = (!p.dense && tid < C) ? p.idx[(size_t)g * C + tid] : 0;
     constexpr int kKRowVecs = D * E::kBytes / 16;   // 16-byte pieces of a key row
-    uint4 kv_app = make_uint4(0u, 0u, 0u, 0u);
-    if (app_i >= 0 && tid < kKRowVecs)
-        kv_app = ldg_stream16(reinterpret_cast<const uint8_t*>(p.k) +
-                              (kv_row_of(p, row / p.hkv, g, row_tok, s - 1) * D) * E::kBytes + tid * 16);
+    uint4 kv_app = make_uint4(0u, 0u, 0u, 0u), vv_app = make_uint4(0u, 0u, 0u, 0u);
+    if (app_i >= 0 && tid < kKRowVecs) {
+        if (p.k_new) {
+            kv_app = ldg_stream16(reinterpret_cast<const uint8_t*>(p.k_new) + ((size_t)row * D) * E::kBytes + tid * 16);
+            vv_app = ldg_stream16(reinterpret_cast<const uint8_t*>(p.v_new) + ((size_t)row * D) * E::kBytes + tid * 16);
+        } else {
+            kv_app = ldg_stream16(reinterpret_cast<const uint8_t*>(p.k) +
+                                  (kv_row_of(p, row / p.hkv, g, row_tok, s - 1) * D) * E::kBytes + tid * 16);
+        }
+    }
 
     // fp label rows stream through a kLabStages-deep shared-memory ring with
     // cp.async (no registers held while in flight): in stage j, thread tid
@@ -340,9 +358,18 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
 #pragma unroll
     for (int e = 0; e < kQPer; ++e)
         if (tid + kNT * e < G * D) qs[tid + kNT * e] = qv[e];
-    // the newest token's key row is staged in `co` (unused until the end)
-    uint8_t* krow_s = reinterpret_cast<uint8_t*>(co);
-    if (app_i >= 0 && tid < kKRowVecs) reinterpret_cast<uint4*>(krow_s)[tid] = kv_app;
+    // the newest token's key row is staged in the bucket list (unused until
+    // the selection; a decode step always has one)
+    uint8_t* krow_s = reinterpret_cast<uint8_t*>(blist);
+    if (app_i >= 0 && tid < kKRowVecs) {
+        reinterpret_cast<uint4*>(krow_s)[tid] = kv_app;
+        if (p.k_new) {  // the new token's K/V rows into the caches (read back by the attention)
+            const size_t r = kv_row_of(p, row / p.hkv, g, row_tok, s - 1) * D * E::kBytes;
+            reinterpret_cast<uint4*>(const_cast<uint8_t*>(reinterpret_cast<const uint8_t*>(p.k)) + r)[tid] = kv_app;
+            reinterpret_cast<uint4*>(const_cast<uint8_t*>(reinterpret_cast<const uint8_t*>(p.v)) + r)[tid] = vv_app;
+            __threadfence();
+        }
+    }
     if (!p.dense) {
         if (tid < C) idx_s[tid] = min(max(iv, 0), D - 1);
         histA[tid] = 0u;
@@ -511,9 +538,9 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         T16 = (bA << 8) | ctl[kCtlBin];
         const int needB = ctl[kCtlNeed];
         refine = needB < ctl[kCtlCnt];
-        // a single-CTA row whose split bucket has at most kNT tokens ranks
-        // them exactly instead of running two more radix passes
-        const bool rank_mode = N == 1 && ctl[kCtlCnt] <= kNT;
+        // a split bucket of at most kNT tokens (over the cluster) is ranked
+        // exactly instead of running two more radix passes
+        const bool rank_mode = ctl[kCtlCnt] <= kNT;
         // Warp w owns the contiguous key groups [wg0, wg1) for the refine
         // sweep and the compaction; in each step lane l reads group
         // wg0 + 32*step + l (conflict-free), so lane order is index order.
@@ -555,21 +582,51 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         if (refine && rank_mode) {
             // rank of each bucket token by (low key bits desc, index asc); the
             // needB-th gives the low threshold, and the tokens equal to it that
-            // rank inside are the ties to take
-            __syncthreads();
-            const int nbl = ctl[kCtlBL];
-            int my_low = -1, my_rank = 0;
-            if (tid < nbl) {
-                const uint32_t e = blist[tid];
-                my_low = (int)(e & 0xFFFFu);
-                const int my_idx = (int)(e >> 16);
-                for (int j = 0; j < nbl; ++j) {
-                    const uint32_t f = blist[j];
-                    const int lo = (int)(f & 0xFFFFu), ix = (int)(f >> 16);
-                    my_rank += (lo > my_low) || (lo == my_low && ix < my_idx);
+            // rank inside are the ties to take. A cluster first gathers every
+            // CTA's bucket list (low key in histB, token index in the row in
+            // histA; both free by now), so all its CTAs rank the same list.
+            int nbl, my_low = -1, my_rank = 0;
+            if (N == 1) {
+                __syncthreads();
+                nbl = ctl[kCtlBL];
+                if (tid < nbl) {
+                    const uint32_t e = blist[tid];
+                    my_low = (int)(e & 0xFFFFu);
+                    const int my_idx = (int)(e >> 16);
+                    for (int j = 0; j < nbl; ++j) {
+                        const uint32_t f = blist[j];
+                        const int lo = (int)(f & 0xFFFFu), ix = (int)(f >> 16);
+                        my_rank += (lo > my_low) || (lo == my_low && ix < my_idx);
+                    }
                 }
-                if (my_rank == needB - 1) ctl[kCtlTlo] = my_low;
+            } else {
+                row_sync(cluster, N);                                // bucket lists complete
+                if (wid == 0) {
+                    const int c = lane < N ? row_smem(cluster, N, ctl, lane)[kCtlBL] : 0;
+                    const int incl = (int)warp_incl_scan((uint32_t)c);
+                    if (lane < N) ctl[kCtlGather + lane] = incl - c;
+                    if (lane == N - 1) ctl[kCtlGather + 16] = incl;
+                }
+                __syncthreads();
+                nbl = min(ctl[kCtlGather + 16], kNT);
+                if (tid < nbl) {
+                    int r = 0;
+                    while (r + 1 < N && ctl[kCtlGather + r + 1] <= tid) ++r;
+                    const uint32_t e = row_smem(cluster, N, blist, r)[tid - ctl[kCtlGather + r]];
+                    histB[tid] = e & 0xFFFFu;
+                    histA[tid] = (uint32_t)(r * p.chunk) + (e >> 16);
+                }
+                __syncthreads();
+                if (tid < nbl) {
+                    my_low = (int)histB[tid];
+                    const int my_idx = (int)histA[tid];
+                    for (int j = 0; j < nbl; ++j) {
+                        const int lo = (int)histB[j], ix = (int)histA[j];
+                        my_rank += (lo > my_low) || (lo == my_low && ix < my_idx);
+                    }
+                }
             }
+            if (tid < nbl && my_rank == needB - 1) ctl[kCtlTlo] = my_low;
             __syncthreads();
             Tlo = ctl[kCtlTlo];
             if (tid < nbl && my_low == Tlo && my_rank < needB) atomicAdd(&ctl[kCtlTie], 1);
@@ -680,38 +737,43 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
             if (lane == 0) scan[wid] = (ns << 16) | nt;
         }
         __syncthreads();
-        if (wid == 0) {
-            const uint32_t x = lane < kNW ? scan[lane] : 0u;
-            const uint32_t xi = warp_incl_scan(x);
-            __syncwarp();
-            if (lane < kNW) scan[lane] = xi - x;
-            if (lane == kNW - 1) { ctl[kCtlCS] = (int)(xi >> 16); ctl[kCtlCT] = (int)(xi & 0xFFFFu); }
+        // each warp's (selected, tie) counts before it and the CTA's totals,
+        // from the kNW per-warp counts
+        uint32_t before = 0, all = 0;
+#pragma unroll
+        for (int w = 0; w < kNW; ++w) {
+            const uint32_t x = scan[w];
+            before += w < wid ? x : 0u;
+            all += x;
         }
         // [phase] 16
-        // [phase] 17
-        if (N > 1) row_sync(cluster, N);                             // per-CTA counts visible
-        // [phase] 18
-        if (N == 1) {
-            if (tid == 0) { ctl[kCtlP] = 0; ctl[kCtlTP] = 0; }
-        } else if (wid == 0) {
-            int cs = 0, ct = 0;
-            if (lane < N) {
-                const int* rc = row_smem(cluster, N, ctl, lane);
-                cs = rc[kCtlCS];
-                ct = rc[kCtlCT];
+        int P = 0, TP = 0;  // selections and ties of the cluster's CTAs before this one
+        if (N > 1) {
+            if (tid == 0) { ctl[kCtlCS] = (int)(all >> 16); ctl[kCtlCT] = (int)(all & 0xFFFFu); }
+            // [phase] 17
+            row_sync(cluster, N);                                    // per-CTA counts visible
+            // [phase] 18
+            if (wid == 0) {
+                int cs = 0, ct = 0;
+                if (lane < N) {
+                    const int* rc = row_smem(cluster, N, ctl, lane);
+                    cs = rc[kCtlCS];
+                    ct = rc[kCtlCT];
+                }
+                const int tp_incl = (int)warp_incl_scan((uint32_t)ct);
+                const int tp = tp_incl - ct;  // ties in CTAs before `lane`
+                const int ntake = refine ? max(0, min(ct, r_tie - tp)) : 0;
+                const int cnt = cs + ntake;
+                const int p_incl = (int)warp_incl_scan((uint32_t)cnt);
+                if (lane == rank) { ctl[kCtlP] = p_incl - cnt; ctl[kCtlTP] = tp; }
             }
-            const int tp_incl = (int)warp_incl_scan((uint32_t)ct);
-            const int tp = tp_incl - ct;  // ties in CTAs before `lane`
-            const int ntake = refine ? max(0, min(ct, r_tie - tp)) : 0;
-            const int cnt = cs + ntake;
-            const int p_incl = (int)warp_incl_scan((uint32_t)cnt);
-            if (lane == rank) { ctl[kCtlP] = p_incl - cnt; ctl[kCtlTP] = tp; }
+            __syncthreads();
+            P = ctl[kCtlP];
+            TP = ctl[kCtlTP];
         }
-        __syncthreads();
         // [phase] 19
-        const int P = ctl[kCtlP], TP = ctl[kCtlTP];
         const int tie_quota = max(0, r_tie - TP);  // ties this CTA may still take
-        int sb = (int)(scan[wid] >> 16), tb = (int)(scan[wid] & 0xFFFFu);  // before this step
+        int sb = (int)(before >> 16), tb = (int)(before & 0xFFFFu);  // before this step
         const uint32_t per = (uint32_t)p.per;
         const uint32_t per_inv = 0xFFFFFFFFu / per;  // q = umulhi(pos, per_inv) is q or q-1
         int cur_dst = -1;
@@ -1023,7 +1085,15 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     else
         attend([&](int j) -> size_t { return row_tok + (size_t)(select_all ? t0 + j : sel_list[j]); });
     __syncthreads();
-    // merge the warps' states per head; a single-CTA row writes its output here
+    // merge the warps' states per head; a single-CTA row writes its output
+    // here. In a cluster, CTA o owns the output elements [o*slice, ...): every
+    // CTA pushes its partial o of those elements, and its (m, l) per head, into
+    // the owner's shared memory (remote stores, no waiting), and after one
+    // cluster barrier each owner merges its slice from local memory.
+    const int slice = (G * D + N - 1) / N;
+    // remote shared memory may only be written once every CTA of the cluster
+    // is running: rows that skipped the selection have had no cluster barrier yet
+    if (N > 1 && select_all) row_sync(cluster, N);
     for (int e = tid; e < G * D; e += kNT) {
         const int h = e / D, d = e - h * D;
         float M = -INFINITY;
@@ -1044,32 +1114,33 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         if (N == 1) {
             write_out(h, d, O / Lsum);
         } else {
-            co[h * D + d] = O;
-            if (d == 0) { cm[h] = M; cl[h] = Lsum; }
+            const int own = e / slice;
+            row_smem(cluster, N, co, own)[rank * slice + (e - own * slice)] = O;
+            if (d == 0)
+                for (int r = 0; r < N; ++r) {
+                    row_smem(cluster, N, cm, r)[rank * GT + h] = M;
+                    row_smem(cluster, N, cl, r)[rank * GT + h] = Lsum;
+                }
         }
     }
     if (N > 1) {
         // [phase] 8
-        row_sync(cluster, N);                                        // CTA partials visible
-        // final merge across the cluster; CTA `rank` writes its slice of [G, D]
-        const int E_all = G * D;
-        const int slice = (E_all + N - 1) / N;
-        const int e0 = rank * slice, e1 = min(E_all, e0 + slice);
+        row_sync(cluster, N);                                        // all partials delivered
+        const int e0 = rank * slice, e1 = min(G * D, e0 + slice);
         for (int e = e0 + tid; e < e1; e += kNT) {
             const int h = e / D, d = e - h * D;
             float M = -INFINITY;
-            for (int r = 0; r < N; ++r) M = fmaxf(M, row_smem(cluster, N, cm, r)[h]);
+            for (int r = 0; r < N; ++r) M = fmaxf(M, cm[r * GT + h]);
             float O = 0.f, Lsum = 0.f;
             for (int r = 0; r < N; ++r) {
-                const float mr = row_smem(cluster, N, cm, r)[h];
+                const float mr = cm[r * GT + h];
                 if (mr == -INFINITY) continue;
                 const float f = exp2f(mr - M);
-                O = fmaf(f, row_smem(cluster, N, co, r)[h * D + d], O);
-                Lsum = fmaf(f, row_smem(cluster, N, cl, r)[h], Lsum);
+                O = fmaf(f, co[r * slice + (e - e0)], O);
+                Lsum = fmaf(f, cl[r * GT + h], Lsum);
             }
             write_out(h, d, O / Lsum);
         }
-        row_sync(cluster, N);                                        // keep smem alive for readers
     }
     // [phase] 9
 }

@@ -214,6 +214,21 @@ DS_API ds_status ds_decode_step(const void* q, const void* k, const void* v, ds_
                                 float sm_scale, void* out, ds_dtype out_dt,
                                 int32_t* sel_out, float* score_out, cudaStream_t stream);
 
+/* ds_decode_step that also takes the new token's key and value rows,
+ * k_new and v_new [b, hkv, d] (dtype kvdt, device or device-mapped, 16-byte
+ * aligned), and writes them into k and v at position s-1 itself before using
+ * them: the serving loop then needs one host-to-device copy (q, k_new, v_new
+ * side by side) and this one launch per layer and step. Otherwise the same
+ * arguments and results as ds_decode_step with those rows already in the
+ * caches. DS_ERR_INVALID_ARG if k_new or v_new is NULL. */
+DS_API ds_status ds_decode_step_kv(const void* q, const void* k_new, const void* v_new,
+                                   void* k, void* v, ds_dtype kvdt,
+                                   void* label, ds_dtype label_dt,
+                                   uint16_t* lscale, uint16_t* lzero, const int32_t* idx,
+                                   int b, int hq, int hkv, int s, int s_cap, int d, int c, int topk,
+                                   float sm_scale, void* out, ds_dtype out_dt,
+                                   int32_t* sel_out, float* score_out, cudaStream_t stream);
+
 /* When a batch entry is decoded with every one of its tokens instead of its
  * top-k (the pages' SGLang section: --ds-sparse-decode-threshold and the
  * heavy-token count decide when Double Sparsity is not used).

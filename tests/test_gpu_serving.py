@@ -7,6 +7,7 @@
 - key/value caches in pinned host memory read by the kernels over the host
   link (Double Sparsity's offloading mode), bit-identical to device caches;
 - paged K/V pools with a block table, bit-identical to the dense layout;
+- the decode step that writes the new token's K/V rows itself;
 - the channel criteria of ds_calibrate_channels_criterion (Q-, K-, QK-outlier,
   chunked QK norm, LeanK ratio): channel indices bit-exact.
 """
@@ -399,3 +400,45 @@ def test_paged_rejects_bad_tables():
                              lab, idx, table, 40, 16)
     ds.decode_step_paged(q, pool, pool, lab, idx, table, 64, 16)   # valid
     torch.cuda.synchronize()
+
+
+# -------------------------------------------- new token's rows in the launch
+
+@pytest.mark.parametrize("kv,label,cluster", [("bf16", "bf16", 0), ("bf16", "int4", 4), ("f32", "f32", 2),
+                                              ("bf16", "bf16", 16)])
+def test_decode_step_kv_equals_copy_then_step(kv, label, cluster):
+    """ds_decode_step_kv writes the new token's K/V rows into the caches and
+    then runs the step: the same bits as copying them in and calling
+    ds_decode_step (caches, label cache, selection, output)."""
+    b, hq, hkv, d, c, s, topk = 3, 8, 4, 128 if kv == "bf16" else 64, 16, 5000, 300
+    if label == "int4":
+        c = 32
+    if kv == "f32":
+        c = 8
+    wl = synth.custom(b=b, hq=hq, hkv=hkv, d=d, s=s, c=c, topk=topk, kv_dtype=kv, label_dtype=label,
+                      n_outlier=min(16, c), outlier_scale=6.0, index=86)
+    di = synth.decode_inputs(wl, s_cap=s + 8)
+    idx = _idx_random(wl, 14)
+    qd, kd, vd = (to_dev(x, kv) for x in (di.q, di.k, di.v))
+    idxd = torch.from_numpy(idx).cuda()
+    k_new, v_new = kd[:, :, s - 1].clone(), vd[:, :, s - 1].clone()
+    k1, v1 = kd.clone(), vd.clone()
+    k1[:, :, s - 1] = 0
+    v1[:, :, s - 1] = 0
+    lab1, sc1, ze1 = _label_alloc(kd, wl)
+    ds.build_label_cache(kd, idxd, s - 1, lab1, sc1, ze1)
+    lab2 = lab1.clone()
+    sc2, ze2 = (None, None) if sc1 is None else (sc1.clone(), ze1.clone())
+    sel1 = torch.empty((b, hkv, topk), dtype=torch.int32, device="cuda")
+    sel2 = torch.empty_like(sel1)
+    ds.set_cluster(cluster)
+    try:
+        o1 = ds.decode_step_kv(qd, k_new, v_new, k1, v1, lab1, idxd, s, topk, lscale=sc1, lzero=ze1, sel_out=sel1)
+        o2 = ds.decode_step(qd, kd, vd, lab2, idxd, s, topk, lscale=sc2, lzero=ze2, sel_out=sel2)
+        torch.cuda.synchronize()
+    finally:
+        ds.set_cluster(0)
+    assert torch.equal(k1, kd) and torch.equal(v1, vd)
+    assert torch.equal(lab1, lab2) and torch.equal(sel1, sel2) and torch.equal(o1, o2)
+    if sc1 is not None:
+        assert torch.equal(sc1, sc2) and torch.equal(ze1, ze2)
