@@ -142,7 +142,12 @@ cudaError_t prepare_kernel(ds::DecodeKernel kern, int smem, int N) {
     return cudaSuccess;
 }
 
-ds::DecodeKernel pick_kernel(ds_dtype kvdt, bool int4, int d, int c, int GT) {
+ds::DecodeKernel pick_kernel(ds_dtype kvdt, bool int4, int d, int c, int GT, bool paged = false) {
+    if (paged) {
+        if (kvdt == DS_F32)
+            return int4 ? ds::decode_kernel_f32_i4_paged(d, c, GT) : ds::decode_kernel_f32_fp_paged(d, c, GT);
+        return int4 ? ds::decode_kernel_bf16_i4_paged(d, c, GT) : ds::decode_kernel_bf16_fp_paged(d, c, GT);
+    }
     if (kvdt == DS_F32) return int4 ? ds::decode_kernel_f32_i4(d, c, GT) : ds::decode_kernel_f32_fp(d, c, GT);
     return int4 ? ds::decode_kernel_bf16_i4(d, c, GT) : ds::decode_kernel_bf16_fp(d, c, GT);
 }
@@ -411,7 +416,7 @@ ds_status sparse_decode_impl(const void* q, const void* k, const void* v, ds_dty
                    kCtasPerSm * sm_count(),
                    g_cluster_override.load(), &pl))
         return fail(DS_ERR_UNSUPPORTED, "no feasible launch plan (s too long for 16 CTAs per row)");
-    ds::DecodeKernel kern = pick_kernel(kvdt, label_dt == DS_INT4, d, c, GT);
+    ds::DecodeKernel kern = pick_kernel(kvdt, label_dt == DS_INT4, d, c, GT, pg != nullptr);
     if (!kern) return fail(DS_ERR_UNSUPPORTED, "no kernel for d=%d c=%d G=%d", d, c, G);
     ds::DecodeParams p{};
     if (seq_lens && !aligned16(seq_lens)) return fail(DS_ERR_INVALID_ARG, "seq_lens not 16-byte aligned");

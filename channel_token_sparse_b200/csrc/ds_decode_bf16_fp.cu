@@ -6,7 +6,7 @@ namespace ds {
 
 DecodeKernel decode_kernel_bf16_fp(int D, int C, int GT) {
 #define DS_K(D_, C_, G_) \
-    if (D == D_ && C == C_ && GT == G_) return &ds_decode_kernel<bf16_t, 0, D_, C_, G_>;
+    if (D == D_ && C == C_ && GT == G_) return &ds_decode_kernel<bf16_t, 0, D_, C_, G_, false>;
 #define DS_KG(D_, C_) DS_K(D_, C_, 1) DS_K(D_, C_, 2) DS_K(D_, C_, 4) DS_K(D_, C_, 8)
     DS_KG(64, 8) DS_KG(64, 16) DS_KG(64, 32) DS_KG(64, 64)
     DS_KG(128, 8) DS_KG(128, 16) DS_KG(128, 32) DS_KG(128, 64) DS_KG(128, 128)

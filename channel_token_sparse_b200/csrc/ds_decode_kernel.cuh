@@ -79,8 +79,9 @@ struct DecodeParams {
 
 // Row (in units of d elements) of token t of (b, g) in the K/V caches, dense
 // or paged; block ids are clamped into the pool.
+template <bool PAGED>
 __device__ __forceinline__ size_t kv_row_of(const DecodeParams& p, int b, int g, size_t row_tok, int t) {
-    if (!p.block_table) return row_tok + (size_t)t;
+    if constexpr (!PAGED) return row_tok + (size_t)t;
     int blk = __ldg(p.block_table + (size_t)b * p.max_blocks + (t >> p.page_shift));
     blk = min(max(blk, 0), p.num_blocks - 1);
     return (((size_t)blk * p.hkv + g) << p.page_shift) + (size_t)(t & ((1 << p.page_shift) - 1));
@@ -236,7 +237,9 @@ __device__ __forceinline__ void cluster_select_bin(cg::cluster_group& cluster, u
     __syncthreads();
 }
 
-template <typename TKV, int LK, int D, int C, int GT>
+// PAGED: K/V are paged pools addressed through p.block_table (a separate
+// instantiation, so the dense layout's copy loops carry no lookup).
+template <typename TKV, int LK, int D, int C, int GT, bool PAGED>
 __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p) {
     using E = Elem<TKV>;
     using LG = LabelGeom<TKV, LK, C>;
@@ -326,7 +329,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
             vv_app = ldg_stream16(reinterpret_cast<const uint8_t*>(p.v_new) + ((size_t)row * D) * E::kBytes + tid * 16);
         } else {
             kv_app = ldg_stream16(reinterpret_cast<const uint8_t*>(p.k) +
-                                  (kv_row_of(p, row / p.hkv, g, row_tok, s - 1) * D) * E::kBytes + tid * 16);
+                                  (kv_row_of<PAGED>(p, row / p.hkv, g, row_tok, s - 1) * D) * E::kBytes + tid * 16);
         }
     }
 
@@ -364,7 +367,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     if (app_i >= 0 && tid < kKRowVecs) {
         reinterpret_cast<uint4*>(krow_s)[tid] = kv_app;
         if (p.k_new) {  // the new token's K/V rows into the caches (read back by the attention)
-            const size_t r = kv_row_of(p, row / p.hkv, g, row_tok, s - 1) * D * E::kBytes;
+            const size_t r = kv_row_of<PAGED>(p, row / p.hkv, g, row_tok, s - 1) * D * E::kBytes;
             reinterpret_cast<uint4*>(const_cast<uint8_t*>(reinterpret_cast<const uint8_t*>(p.k)) + r)[tid] = kv_app;
             reinterpret_cast<uint4*>(const_cast<uint8_t*>(reinterpret_cast<const uint8_t*>(p.v)) + r)[tid] = vv_app;
             __threadfence();
@@ -825,9 +828,9 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     // paged K/V: this CTA's selected tokens become pool rows first (one
     // table lookup per token, all in flight together)
     uint32_t* sel_rows = reinterpret_cast<uint32_t*>(sel_list);
-    if (p.block_table && !select_all) {
+    if (PAGED && !select_all) {
         for (int j = tid; j < n_att; j += kNT)
-            sel_rows[j] = (uint32_t)kv_row_of(p, row / p.hkv, g, row_tok, sel_list[j]);
+            sel_rows[j] = (uint32_t)kv_row_of<PAGED>(p, row / p.hkv, g, row_tok, sel_list[j]);
         __syncthreads();
     }
     float* wp_out = nullptr;  // this warp's partial (m, l, o) per head, [GT][D + 2]
@@ -836,11 +839,14 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         if (p.out_bf16) reinterpret_cast<uint16_t*>(p.out)[oidx] = f32_to_bf16_bits(res);
         else reinterpret_cast<float*>(p.out)[oidx] = res;
     };
-    // The attention phase, instantiated once per K/V addressing (dense
-    // caches, or paged pools through the block table) so that the row lookup
-    // adds no branch to the copy loops. att_row(j) is the K/V row (units of d
-    // elements) of the j-th token this CTA attends.
-    auto attend = [&](auto att_row) {
+    // K/V row (units of d elements) of the j-th token this CTA attends
+    auto att_row = [&](int j) -> size_t {
+        if constexpr (PAGED)
+            return select_all ? kv_row_of<PAGED>(p, row / p.hkv, g, row_tok, t0 + j) : (size_t)sel_rows[j];
+        else
+            return row_tok + (size_t)(select_all ? t0 + j : sel_list[j]);
+    };
+    {
         if constexpr (E::kBytes == 2) {
             // bf16 K/V: tensor cores (mma.sync, fp32 accumulate) on 8-token tiles.
             //   Z  = Q K^T   m16n8k16: rows = the group's heads (padded to 16),
@@ -1077,13 +1083,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
             }
         }
         }
-    };
-    if (p.block_table)
-        attend([&](int j) -> size_t {
-            return select_all ? kv_row_of(p, row / p.hkv, g, row_tok, t0 + j) : (size_t)sel_rows[j];
-        });
-    else
-        attend([&](int j) -> size_t { return row_tok + (size_t)(select_all ? t0 + j : sel_list[j]); });
+    }
     __syncthreads();
     // merge the warps' states per head; a single-CTA row writes its output
     // here. In a cluster, CTA o owns the output elements [o*slice, ...): every

@@ -15,6 +15,11 @@ DecodeKernel decode_kernel_f32_fp(int D, int C, int GT);
 DecodeKernel decode_kernel_f32_i4(int D, int C, int GT);
 DecodeKernel decode_kernel_bf16_fp(int D, int C, int GT);
 DecodeKernel decode_kernel_bf16_i4(int D, int C, int GT);
+// The same for paged K/V pools (ds_decode_step_paged).
+DecodeKernel decode_kernel_f32_fp_paged(int D, int C, int GT);
+DecodeKernel decode_kernel_f32_i4_paged(int D, int C, int GT);
+DecodeKernel decode_kernel_bf16_fp_paged(int D, int C, int GT);
+DecodeKernel decode_kernel_bf16_i4_paged(int D, int C, int GT);
 
 struct LabelArgs {
     const void* k;
