@@ -572,15 +572,34 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
                 mcache[grp] = (uint16_t)above;   // keys selected outright, for the write pass
                 for (uint32_t m = flags; m; m &= m - 1) {
                     const int i = grp * 8 + __ffs(m) - 1;
-                    const uint32_t low = p.keep_low ? (uint32_t)low16[i] : score_key(rescore(i)) & 0xFFFFu;
-                    keys[i] = (uint16_t)low;
-                    if (!rank_mode) atomicAdd(&histA[low >> 8], 1u);
                     const int slot = atomicAdd(&ctl[kCtlBL], 1);
-                    if (slot < kBucketCap) blist[slot] = low | ((uint32_t)i << 16);
+                    if (p.keep_low || slot >= kBucketCap) {
+                        // low bits at hand, or no list slot left: take them here
+                        const uint32_t low = p.keep_low ? (uint32_t)low16[i] : score_key(rescore(i)) & 0xFFFFu;
+                        keys[i] = (uint16_t)low;
+                        if (!rank_mode) atomicAdd(&histA[low >> 8], 1u);
+                        if (slot < kBucketCap) blist[slot] = low | ((uint32_t)i << 16);
+                    } else {
+                        blist[slot] = (uint32_t)i << 16;  // re-scored below
+                    }
                 }
             }
             above_cnt = __reduce_add_sync(0xffffffffu, above_cnt);
             if (lane == 0) ctl[kCtlWarp + wid] = (int)(above_cnt << 16);
+            if (!p.keep_low) {
+                // the listed bucket tokens are re-scored all at once (one
+                // label-row load per thread in flight, not one per lane in turn)
+                __syncthreads();
+                const int nbl = min(ctl[kCtlBL], kBucketCap);
+                for (int j = tid; j < nbl; j += kNT) {
+                    const uint32_t e = blist[j];
+                    const int i = (int)(e >> 16);
+                    const uint32_t low = score_key(rescore(i)) & 0xFFFFu;
+                    keys[i] = (uint16_t)low;
+                    blist[j] = e | low;
+                    if (!rank_mode) atomicAdd(&histA[low >> 8], 1u);
+                }
+            }
         }
         if (refine && rank_mode) {
             // rank of each bucket token by (low key bits desc, index asc); the
