@@ -168,18 +168,22 @@ __device__ __forceinline__ float label_score(const uint32_t (&w)[LabelGeom<TKV, 
     auto ql = [&](int j) -> float { return kReg ? qreg[j] : qsm[j]; };
     float acc = 0.f;
     if constexpr (LK == kLabelInt4) {
+        // Nibble e of a word holds channel e. Shifted to bits 19..22 (the
+        // top of the mantissa) and or-ed into 1.0f it gives 1 + n/16 exactly,
+        // so a nibble costs a shift, a mask and an FMA (no conversion):
+        //   sum_j qL[j] n_j = 16 (sum_j qL[j] (1 + n_j/16) - sum_j qL[j])
 #pragma unroll
         for (int i = 0; i < C / 8; ++i) {
             const uint32_t x = w[i];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                // nibble -> float exactly: 2^23 + n has n in its low mantissa bits
-                const float n = __uint_as_float(0x4B000000u | ((x >> (4 * e)) & 15u)) - 8388608.0f;
-                acc = __fmaf_rn(ql(8 * i + e), n, acc);
+                const uint32_t t = 4 * e <= 19 ? (x << (19 - 4 * e)) : (x >> (4 * e - 19));
+                acc = __fmaf_rn(ql(8 * i + e), __uint_as_float((t & 0x00780000u) | 0x3F800000u), acc);
             }
         }
+        const float dot = __fmul_rn(16.f, __fsub_rn(acc, qsum));
         // sum_j qL[j] * (sc * n_j + z) = sc * sum_j qL[j] n_j + z * sum_j qL[j]
-        return __fmaf_rn(sc, acc, __fmul_rn(z, qsum));
+        return __fmaf_rn(sc, dot, __fmul_rn(z, qsum));
     } else if constexpr (Elem<TKV>::kBytes == 2) {
 #pragma unroll
         for (int i = 0; i < C / 2; ++i) {
