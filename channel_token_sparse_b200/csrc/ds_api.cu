@@ -75,7 +75,7 @@ int round_up(int x, int m) { return (x + m - 1) / m * m; }
 // least 256 tokens per CTA; rows beyond one wave use N = 1. A forced N
 // (ds_sparse_decode_set_cluster) overrides the choice when feasible.
 bool make_plan(int rows, int G, int s, int d, int c, int topk, bool dense, bool int4, int esz, int slots,
-               int forced, Plan* out) {
+               int forced, Plan* out, int s_cap = 0) {
     const int GT = group_tier(G);
     const bool select_all = dense || topk >= s;
     const int k_eff = topk < s ? topk : s;
@@ -104,14 +104,23 @@ bool make_plan(int rows, int G, int s, int d, int c, int topk, bool dense, bool 
             const ds::DecodeSmem L = ds::decode_smem_layout(GT, d, c, p.lay_chunk, p.per, esz, p.att_stages);
             const int region = L.total - L.region;
             const int keys = ds::align16(p.lay_chunk * 2);
-            const int ring = (!int4 && (c * esz) % 16 == 0) ? ds::lab_ring_bytes(c * esz) : -1;
+            // 4-bit rows also stream their fp16 scale and zero in 16-byte
+            // chunks of 8 tokens, which needs rows of a multiple of 8 tokens
+            const int pay = c / 2;
+            const bool i4_ring = int4 && s_cap > 0 && s_cap % 8 == 0 && (pay == 4 || pay == 8 || pay % 16 == 0);
+            const int ring = int4 ? (i4_ring ? ds::lab_ring_bytes(pay + 4) : -1)
+                                  : ((c * esz) % 16 == 0 ? ds::lab_ring_bytes(c * esz) : -1);
+            // (for 4-bit rows, whose re-scoring costs more, the kept low
+            // bits come before the ring when only one of them fits)
             if (ring >= 0 && 2 * keys + ring <= region) {
                 p.lab_ring = 1;
                 p.keep_low = 1;
-            } else if (ring >= 0 && keys + ring <= region) {
+            } else if (ring >= 0 && keys + ring <= region && !int4) {
                 p.lab_ring = 1;
             } else if (2 * keys <= region) {
                 p.keep_low = 1;
+            } else if (ring >= 0 && keys + ring <= region) {
+                p.lab_ring = 1;
             }
         }
         if (forced) {
@@ -414,7 +423,7 @@ ds_status sparse_decode_impl(const void* q, const void* k, const void* v, ds_dty
     Plan pl;
     if (!make_plan(rows, G, s, d, c, topk, false, label_dt == DS_INT4, kvdt == DS_F32 ? 4 : 2,
                    kCtasPerSm * sm_count(),
-                   g_cluster_override.load(), &pl))
+                   g_cluster_override.load(), &pl, s_cap))
         return fail(DS_ERR_UNSUPPORTED, "no feasible launch plan (s too long for 16 CTAs per row)");
     ds::DecodeKernel kern = pick_kernel(kvdt, label_dt == DS_INT4, d, c, GT, pg != nullptr);
     if (!kern) return fail(DS_ERR_UNSUPPORTED, "no kernel for d=%d c=%d G=%d", d, c, G);

@@ -103,6 +103,8 @@ __host__ __device__ inline int align16(int x) { return (x + 15) & ~15; }
 constexpr int kAttStagesF32 = 4;
 // Label-streaming ring (fp labels): stages of one row per thread.
 constexpr int kLabStages = 8;
+// ring bytes for label rows of `label_row_bytes` (a 4-bit row adds its fp16
+// scale and zero, 4 bytes, kept in two arrays of the stage)
 __host__ __device__ constexpr int lab_ring_bytes(int label_row_bytes) { return kLabStages * 256 * label_row_bytes; }
 __host__ __device__ constexpr int att_stage_tokens(int row_bytes, int elem_bytes) {
     return elem_bytes == 2 ? 8 : (row_bytes >= 1024 ? 1 : 1024 / row_bytes);
@@ -341,20 +343,40 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     // cp.async (no registers held while in flight): in stage j, thread tid
     // copies and then scores local token j * kNT + tid, so it only ever reads
     // its own copies (no block barrier needed).
-    constexpr bool kRingable = LK == kLabelFp && LG::kBytes % 16 == 0;
+    // A 4-bit stage is [256 payloads][256 scales][256 zeros]; the scales and
+    // zeros of warp w's 32 tokens are 4 + 4 16-byte chunks, copied by lanes
+    // 0..7 of that warp (so a __syncwarp makes them visible to its lanes).
+    constexpr bool kI4 = LK == kLabelInt4;
+    constexpr bool kRingable = kI4 ? (LG::kBytes == 4 || LG::kBytes == 8 || LG::kBytes % 16 == 0)
+                                   : LG::kBytes % 16 == 0;
     const bool use_ring = kRingable && need_scores && p.lab_ring;
     uint16_t* low16 = reinterpret_cast<uint16_t*>(smem + L.region + align16(p.lay_chunk * 2));
     uint8_t* lring = smem + L.region + align16(p.lay_chunk * 2) * (p.keep_low ? 2 : 1);
-    constexpr int kSlot = LG::kBytes;               // bytes per token
-    constexpr int kStage = kNT * kSlot;
+    constexpr int kSlot = LG::kBytes;               // payload bytes per token
+    constexpr int kStage = kNT * (kSlot + (kI4 ? 4 : 0));
     const int nst = (n_loc + kNT - 1) / kNT;
     auto issue = [&](int j) {
         const int i = j * kNT + tid;
+        uint8_t* stg = lring + (j % kLabStages) * kStage;
         if (j < nst && i < n_loc && i != app_i) {
-            uint8_t* dst = lring + (j % kLabStages) * kStage + tid * kSlot;
+            uint8_t* dst = stg + tid * kSlot;
             const uint8_t* src = lab + (size_t)(t0 + i) * kSlot;
+            if constexpr (kSlot % 16 == 0) {
 #pragma unroll
-            for (int o = 0; o < kSlot; o += 16) cp_async16(dst + o, src + o);
+                for (int o = 0; o < kSlot; o += 16) cp_async16(dst + o, src + o);
+            } else if constexpr (kSlot == 8) {
+                cp_async8(dst, src);
+            } else {
+                cp_async4(dst, src);
+            }
+        }
+        if constexpr (kI4) {
+            const int c8 = (wid * 32 + (lane & 3) * 8);   // first token of this lane's chunk
+            if (j < nst && lane < 8 && j * kNT + c8 < n_loc) {
+                const uint16_t* src = (lane < 4 ? lsc : lze) + t0 + j * kNT + c8;
+                uint8_t* dst = stg + kNT * kSlot + (lane < 4 ? 0 : kNT * 2) + c8 * 2;
+                cp_async16(dst, src);
+            }
         }
     };
     if (use_ring) {
@@ -477,15 +499,27 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     if (use_ring) {
 #pragma unroll 1
         for (int j = 0; j < nst; ++j) {
+            if constexpr (kI4) __syncwarp();   // every lane is done with the slot refilled next
             issue(j + kLabStages - 1);
             cp_async_commit();
             cp_async_wait<kLabStages - 1>();
+            if constexpr (kI4) __syncwarp();   // the warp's scale / zero chunks
             const int i = j * kNT + tid;
             if (i < n_loc) {
                 uint32_t w[LG::kWords];
-                if (i == app_i) lds_row<LG::kBytes>(w, app_row);
-                else lds_row<LG::kBytes>(w, lring + (j % kLabStages) * kStage + tid * kSlot);
-                score_token(i, w, 0.f, 0.f);
+                const uint8_t* stg = lring + (j % kLabStages) * kStage;
+                float ss = 0.f, zz = 0.f;
+                if (i == app_i) {
+                    lds_row<LG::kBytes>(w, app_row);
+                    if constexpr (kI4) { ss = fp16_bits_to_f32(app_sz[0]); zz = fp16_bits_to_f32(app_sz[1]); }
+                } else {
+                    lds_row<LG::kBytes>(w, stg + tid * kSlot);
+                    if constexpr (kI4) {
+                        ss = fp16_bits_to_f32(reinterpret_cast<const uint16_t*>(stg + kNT * kSlot)[tid]);
+                        zz = fp16_bits_to_f32(reinterpret_cast<const uint16_t*>(stg + kNT * kSlot + kNT * 2)[tid]);
+                    }
+                }
+                score_token(i, w, ss, zz);
             }
         }
         cp_async_wait<0>();
