@@ -585,7 +585,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         // Warp w owns the contiguous key groups [wg0, wg1) for the refine
         // sweep and the compaction; in each step lane l reads group
         // wg0 + 32*step + l (conflict-free), so lane order is index order.
-        const int gpw = (((ngrp + kNW - 1) / kNW) + 31) & ~31;   // groups per warp
+        const int gpw = (((ngrp + kNW - 1) / kNW) + 63) & ~63;   // groups per warp
         const int wg0 = wid * gpw, wg1 = min(ngrp, wg0 + gpw);
         // [phase] 4
         if (refine) {
@@ -838,9 +838,14 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         const uint32_t per_inv = 0xFFFFFFFFu / per;  // q = umulhi(pos, per_inv) is q or q-1
         int cur_dst = -1;
         int* rl = nullptr;
-        for (int grp = wg0 + lane; grp - lane < wg1; grp += 32) {
-            const uint32_t m = grp < wg1 ? (counts_known ? masks_swept(grp) : (uint32_t)mcache[grp]) : 0u;
-            const uint32_t smk = m & 255u, tmk = m >> 8;
+        // two key groups (16 tokens) per lane and step: lane l takes groups
+        // g0 = wg0 + 64*step + 2l and g0 + 1, so lane order is still index order
+        auto gmask = [&](int grp) -> uint32_t {
+            return grp < wg1 ? (counts_known ? masks_swept(grp) : (uint32_t)mcache[grp]) : 0u;
+        };
+        for (int g0 = wg0 + 2 * lane; g0 - 2 * lane < wg1; g0 += 64) {
+            const uint32_t m0 = gmask(g0), m1 = gmask(g0 + 1);
+            const uint32_t smk = (m0 & 255u) | ((m1 & 255u) << 8), tmk = (m0 >> 8) | ((m1 >> 8) << 8);
             const uint32_t pk = ((uint32_t)__popc(smk) << 16) | (uint32_t)__popc(tmk);
             const uint32_t incl = warp_incl_scan(pk);
             const int my_sb = sb + (int)((incl - pk) >> 16), my_tb = tb + (int)((incl - pk) & 0xFFFFu);
@@ -854,7 +859,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
                 const int t_before = my_tb + __popc(tmk & below);
                 if (((tmk >> e) & 1u) && t_before >= tie_quota) continue;  // tie beyond the quota
                 const uint32_t pos = (uint32_t)(P + s_before + min(t_before, tie_quota));
-                const int t = t0 + grp * 8 + e;
+                const int t = t0 + g0 * 8 + e;
                 if (N == 1) {
                     sel_list[pos] = t;
                 } else {
