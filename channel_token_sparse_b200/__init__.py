@@ -53,6 +53,7 @@ SIGNATURES = {
     "ds_sparse_decode_plan": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, _i, C.POINTER(_i), C.POINTER(_i),
                                    C.POINTER(_i)]),
     "ds_sparse_decode_set_cluster": (None, [_i]),
+    "ds_sparse_decode_workspace": (_i, [_i, _i, _i, _i, _i, _i, _i, C.POINTER(_sz)]),
     "ds_dense_decode": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _i, _vp]),
 }
 
@@ -166,6 +167,13 @@ def plan(b, hq, hkv, s, d, c, topk, kv_dtype=DS_BF16, label_dtype=DS_BF16):
     _check(lib().ds_sparse_decode_plan(b, hq, hkv, s, d, c, topk, kv_dtype, label_dtype,
                                        C.byref(n), C.byref(ch), C.byref(sm)))
     return n.value, ch.value, sm.value
+
+
+def sparse_decode_workspace(b, hq, hkv, s, d, c, topk) -> int:
+    """Device scratch bytes ds_sparse_decode needs for a shape (0: on chip)."""
+    out = C.c_size_t()
+    _check(lib().ds_sparse_decode_workspace(b, hq, hkv, s, d, c, topk, C.byref(out)))
+    return out.value
 
 
 # -------------------------------------------------------------- entry points

@@ -375,6 +375,18 @@ ds_status ds_append_label(const void* k, ds_dtype kdt, const int32_t* idx, int b
                      stream);
 }
 
+ds_status ds_sparse_decode_workspace(int b, int hq, int hkv, int s, int d, int c, int topk,
+                                     size_t* bytes) {
+    if (!bytes) return fail(DS_ERR_INVALID_ARG, "bytes is NULL");
+    ds_status r = check_common(b, hq, hkv, s, s, d, DS_BF16);
+    if (r != DS_OK) return r;
+    if (!c_ok(c, d)) return fail(DS_ERR_UNSUPPORTED, "heavy channels c=%d (supported: 8,16,32,64,128; c <= d)", c);
+    if (topk < 1) return fail(DS_ERR_INVALID_ARG, "topk must be >= 1");
+    // scores, the selection and the softmax partials of a step stay on chip
+    *bytes = 0;
+    return DS_OK;
+}
+
 ds_status ds_sparse_decode_plan(int b, int hq, int hkv, int s, int d, int c, int topk, ds_dtype kvdt,
                                 ds_dtype label_dt, int* cluster_out, int* chunk_out, int* smem_out) {
     ds_status r = check_common(b, hq, hkv, s, s, d, kvdt);

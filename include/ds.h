@@ -201,6 +201,16 @@ DS_API ds_status ds_sparse_decode(const void* q, const void* k, const void* v, d
                            float sm_scale, void* out, ds_dtype out_dt,
                            int32_t* sel_out, float* score_out, cudaStream_t stream);
 
+/* Device scratch ds_sparse_decode needs for a shape, in bytes (host only,
+ * launches nothing). The decode step of 在线前向计算 keeps its per-step
+ * intermediates -- the approximate scores of step 2, the top-k selection of
+ * step 3 and the partial softmax states -- in shared memory of the thread-block
+ * cluster serving each (b, g), so the answer is 0 for every supported shape and
+ * ds_sparse_decode takes no workspace argument. Validates the shape like
+ * ds_sparse_decode (DS_ERR_INVALID_ARG / DS_ERR_UNSUPPORTED, *bytes untouched). */
+DS_API ds_status ds_sparse_decode_workspace(int b, int hq, int hkv, int s, int d, int c, int topk,
+                                            size_t* bytes);
+
 /* One decode step in one launch (Double Sparsity 离线校准 + 在线前向计算):
  * the label row of the newest token, position s-1, whose K/V the caller has
  * already written, is built exactly as ds_append_label builds it and stored

@@ -113,3 +113,20 @@ def test_plan_choices(lib):
         assert ds.plan(8, 32, 32, 4096, 128, 16, 256)[:2] == (16, 256)
     finally:
         ds.set_cluster(0)
+
+
+def test_sparse_decode_workspace(lib):
+    # every supported shape keeps its per-step scratch on chip
+    for shape in [(8, 32, 32, 4096, 128, 16, 256), (32, 32, 32, 16384, 128, 32, 1024),
+                  (4, 32, 8, 32768, 128, 16, 2048), (1, 32, 32, 262144, 128, 16, 16384),
+                  (1, 2, 2, 512, 64, 8, 32)]:
+        assert ds.sparse_decode_workspace(*shape) == 0
+    out = C.c_size_t(12345)
+    for bad, expect in [((1, 30, 8, 512, 64, 8, 32), ds.DS_ERR_INVALID_ARG),   # hq % hkv
+                        ((1, 2, 2, 512, 96, 8, 32), ds.DS_ERR_UNSUPPORTED),    # head_dim
+                        ((1, 2, 2, 512, 64, 12, 32), ds.DS_ERR_UNSUPPORTED),   # channels
+                        ((1, 2, 2, 512, 64, 8, 0), ds.DS_ERR_INVALID_ARG),     # topk
+                        ((1, 2, 2, 0, 64, 8, 32), ds.DS_ERR_INVALID_ARG)]:     # s
+        assert lib.ds_sparse_decode_workspace(*bad, C.byref(out)) == expect
+        assert out.value == 12345  # untouched on failure
+    assert lib.ds_sparse_decode_workspace(1, 2, 2, 512, 64, 8, 32, None) == ds.DS_ERR_INVALID_ARG
