@@ -1,18 +1,24 @@
 """Benchmark of the Double Sparsity decode step on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config I]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config I] [--also I,J,...]
 
 One step = one decode token for every sequence of a layer, in one launch
 (ds_decode_step): the new token's heavy channels are appended to the label
 cache, then query gather, approximate scores, top-k and exact attention over
-the selected K/V rows. The default workload is the
-Llama-2-7B-shaped layer (batch 8, 32 MHA heads, head_dim 128, 4096 cached
-tokens, 16 bf16 heavy channels, top-256). Inputs are seeded synthetic tensors.
+the selected K/V rows. Inputs are seeded synthetic tensors.
 
-Timing: the step captured in a CUDA graph, CUDA events on the launching stream, a 512 MiB
-L2-flushing write before every timed step, max over ranks under torchrun
-(weak scaling: every rank runs its own layer; no collective on the data path).
-Rank 0 prints one JSON line.
+The headline workload is the largest single-GPU one: batch 32, 32 MHA heads,
+head_dim 128, 16384 cached tokens, a 32-channel 4-bit label cache, top-1024
+(873 MB of label, selected K/V and q/out per step). The JSON line nests the
+same record for the other workloads under "configs" (Llama-2-7B layer,
+Llama-3-8B GQA layer, 256K context).
+
+Timing: the step captured in a CUDA graph, K steps back to back between one
+pair of CUDA events on the launching stream, cycling through enough
+independent layer instances that the inputs exceed the L2; max over ranks
+under torchrun (weak scaling: every rank runs its own layer; no collective on
+the data path). Rank 0 prints one JSON line.
 """
 
 from __future__ import annotations
@@ -198,6 +204,20 @@ def job_value(batch_per_rank: int, world: int, steps: int, max_seconds: float) -
 
 # ------------------------------------------------------------ our arm
 
+def heavy_channels(wl: synth.Workload) -> np.ndarray:
+    """idx [Hkv, C] int32: the planted channels, padded (when C is larger)
+    with the lowest unplanted ones, ascending."""
+    planted = synth.outlier_channels(wl)
+    if planted.shape[1] >= wl.c:
+        return np.ascontiguousarray(planted[:, : wl.c], np.int32)
+    full = []
+    for g in range(wl.hkv):
+        have = list(planted[g])
+        extra = [c for c in range(wl.d) if c not in have][: wl.c - len(have)]
+        full.append(sorted(have + extra))
+    return np.asarray(full, np.int32)
+
+
 def build_state(wl: synth.Workload, dev, rank: int):
     import torch
 
@@ -207,14 +227,7 @@ def build_state(wl: synth.Workload, dev, rank: int):
         q, k, v = (_dev(x, wl.kv_dtype, dev) for x in (di.q, di.k, di.v))
     else:
         q, k, v = synth.decode_inputs_torch(wl, dev, seed_offset=rank)
-    idx = torch.from_numpy(np.ascontiguousarray(synth.outlier_channels(wl)[:, : wl.c], np.int32)).to(dev)
-    if idx.shape[1] < wl.c:  # more heavy channels than planted: pad with the next unused ones
-        full = []
-        for g in range(wl.hkv):
-            have = list(synth.outlier_channels(wl)[g])
-            extra = [c for c in range(wl.d) if c not in have][: wl.c - len(have)]
-            full.append(sorted(have + extra))
-        idx = torch.tensor(full, dtype=torch.int32, device=dev)
+    idx = torch.from_numpy(heavy_channels(wl)).to(dev)
     lab, sc, ze = ds.new_label_cache(k, wl.c, int4=wl.label_dtype == "int4")
     return dict(q=q, k=k, v=v, idx=idx, lab=lab, sc=sc, ze=ze)
 
@@ -403,7 +416,7 @@ def run_ours(args, wl, rank, local_rank, world):
                             ds.DS_BF16 if wl.kv_dtype == "bf16" else ds.DS_F32,
                             ds.DS_INT4 if wl.label_dtype == "int4" else
                             (ds.DS_BF16 if wl.kv_dtype == "bf16" else ds.DS_F32)),
-               out_esz=out.element_size(), host=(q, k, v, idx, lab, sc, ze))
+               out_esz=out.element_size(), rows=DeviceRows(wl, q, k, v, idx))
     return res
 
 
@@ -520,72 +533,171 @@ def barrier():
 
 # ------------------------------------------------------------ CPU oracle
 
-def oracle_sample(wl: synth.Workload, host, budget_s: float, max_rows: int | None = None):
-    """Time the CPU oracle on (b, kv head) rows of the same workload until
-    `budget_s` seconds have passed (at least one row). Returns (seconds per
-    full step, rows timed)."""
+class DeviceRows:
+    """Host copies of single (b, kv head) rows of the device-resident
+    workload, fetched on demand (the multi-GB caches are never copied whole)."""
+
+    def __init__(self, wl, q, k, v, idx):
+        self.wl, self.q, self.k, self.v = wl, q, k, v
+        self.idx = idx.cpu().numpy()
+
+    @staticmethod
+    def _np(t):
+        import torch
+        t = t.contiguous().cpu()
+        return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+
+    def row(self, b, g):
+        wl, G = self.wl, self.wl.g
+        return (self._np(self.q[b:b + 1, g * G:(g + 1) * G]), self._np(self.k[b:b + 1, g:g + 1, : wl.s]),
+                self._np(self.v[b:b + 1, g:g + 1, : wl.s]), np.ascontiguousarray(self.idx[g:g + 1]))
+
+
+class SynthRows:
+    """Rows drawn on the host (the reference arm: no GPU, no full workload)."""
+
+    def __init__(self, wl):
+        self.wl = wl
+        self.idx = heavy_channels(wl)
+
+    def row(self, b, g):
+        q, k, v = synth.decode_row_inputs(self.wl, b, g)
+        return q, k, v, np.ascontiguousarray(self.idx[g:g + 1])
+
+
+def oracle_row(wl, row):
+    """One (b, kv head) row of a step on the oracle: label build (prefill and
+    append) and the sparse decode."""
     import oracle
-    q, k, v, idx, lab, sc, ze = host
-    G = wl.g
-    rows = [(b, g) for b in range(wl.b) for g in range(wl.hkv)]
-    done, t_used = 0, 0.0
+    qr, kr, vr, ir = row
+    labr = oracle.build_label(kr, wl.kv_dtype, wl.label_dtype, ir, wl.s)
+    oracle.sparse_decode(qr, kr, vr, wl.kv_dtype, labr, wl.label_dtype, ir, wl.s, wl.topk)
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def _row_list(wl):
+    return [(b, g) for b in range(wl.b) for g in range(wl.hkv)]
+
+
+def oracle_single(wl, rows_src, budget_s: float):
+    """The oracle on one thread, rows in order (each fetched untimed) until
+    `budget_s` seconds of oracle time. Returns (seconds per full step, rows)."""
+    import oracle
+    oracle.build()
+    t_used, done = 0.0, 0
+    rows = _row_list(wl)
     for (b, g) in rows:
-        if max_rows is not None and done >= max_rows:
-            break
-        qr = q[b:b + 1, g * G:(g + 1) * G]
-        kr = np.ascontiguousarray(k[b:b + 1, g:g + 1])
-        vr = np.ascontiguousarray(v[b:b + 1, g:g + 1])
-        ir = np.ascontiguousarray(idx[g:g + 1])
+        row = rows_src.row(b, g)
         t0 = time.perf_counter()
-        labr = oracle.build_label(kr, wl.kv_dtype, wl.label_dtype, ir, wl.s)  # prefill + append
-        oracle.sparse_decode(qr, kr, vr, wl.kv_dtype, labr, wl.label_dtype, ir, wl.s, wl.topk)
+        oracle_row(wl, row)
         t_used += time.perf_counter() - t0
         done += 1
         if t_used >= budget_s:
             break
-    per_row = t_used / done
-    return per_row * len(rows), done
+    return t_used / done * len(rows), done
 
 
-def host_arrays(wl, state_tensors):
-    import torch
-    out = []
-    for t in state_tensors:
-        if t is None:
-            out.append(None)
-        elif t.dtype == torch.bfloat16:
-            out.append(t.view(torch.int16).cpu().numpy().view(np.uint16))
-        elif t.dtype == torch.int16:
-            out.append(t.cpu().numpy().view(np.uint16))
-        else:
-            out.append(t.cpu().numpy())
-    return out
+def oracle_parallel(wl, rows_src, budget_s: float, threads: int, max_bytes: int = 2 << 30):
+    """The oracle on `threads` host threads at once (ctypes releases the GIL
+    while the C code runs). M rows are fetched first (untimed; at most
+    2 * threads and at most `max_bytes` of host copies), then the threads
+    take rows 0, 1, ..., M-1, 0, ... until `budget_s` seconds of wall time.
+    Returns (seconds per full step, rows timed, threads used)."""
+    import concurrent.futures as cf
+    import itertools
+    import oracle
+    oracle.build()
+    oracle._load()  # load once before the threads start
+    esz = 4 if wl.kv_dtype == "f32" else 2
+    row_bytes = 2 * wl.s * wl.d * esz
+    rows = _row_list(wl)
+    m = max(1, min(len(rows), 2 * threads, max_bytes // row_bytes))
+    data = [rows_src.row(b, g) for (b, g) in rows[:m]]
+    used = min(threads, m)
+    counter = itertools.count()
+    t_start = time.perf_counter()
+    deadline = t_start + budget_s
+
+    def worker():
+        n = 0
+        while True:
+            i = next(counter)
+            if n > 0 and time.perf_counter() >= deadline:
+                return n
+            if i >= m and time.perf_counter() >= deadline:
+                return n
+            oracle_row(wl, data[i % m])
+            n += 1
+
+    with cf.ThreadPoolExecutor(max_workers=used) as ex:
+        done = sum(f.result() for f in [ex.submit(worker) for _ in range(used)])
+    wall = time.perf_counter() - t_start
+    return wall / done * len(rows), done, used
+
+
+def cpu_baseline(wl, rows_src, budget_s: float) -> dict:
+    """The oracle timed on this host: all host threads, and one thread."""
+    threads = os.cpu_count() or 1
+    tn, rowsn, used = oracle_parallel(wl, rows_src, budget_s, threads)
+    t1, rows1 = oracle_single(wl, rows_src, budget_s)
+    nrows = wl.b * wl.hkv
+    return {"value": wl.b / tn, "unit": UNIT, "cores": used, "kind": "oracle",
+            "sample": f"{rowsn} (batch, kv-head) rows of one step (label build + scores + top-k + "
+                      f"attention; {nrows} rows per step) on {used} threads for about {budget_s:g} s, "
+                      f"scaled to the full step",
+            "cpu_model": cpu_model(), "host_threads": threads,
+            "single_thread": {"value": wl.b / t1, "unit": UNIT, "cores": 1,
+                              "sample": f"{rows1} of {nrows} rows on 1 thread, scaled to the full step"}}
 
 
 def run_reference(args, wl):
-    """The oracle as the reference arm: each step is a bounded sample (a
-    fixed number of (b, kv head) rows) of the same workload on host cores."""
+    """The oracle as the reference arm: each step is a bounded sample (one
+    (b, kv head) row per host thread, drawn on the host once) of the same
+    workload, processed by all host threads at once."""
+    import concurrent.futures as cf
     import oracle
     oracle.build()
-    di = synth.decode_inputs(wl)
-    idx = np.ascontiguousarray(synth.outlier_channels(wl)[:, : wl.c], np.int32)
-    host = (di.q, di.k, di.v, idx, None, None, None)
-    rows_per_step = max(1, min(wl.b * wl.hkv, args.ref_rows))
-    for _ in range(args.warmup):
-        oracle_sample(wl, host, 0.0, max_rows=rows_per_step)
-    t_total = 0.0
-    for _ in range(args.steps):
+    oracle._load()
+    threads = os.cpu_count() or 1
+    src = SynthRows(wl)
+    rows = _row_list(wl)
+    esz = 4 if wl.kv_dtype == "f32" else 2
+    cap = max(1, (2 << 30) // (2 * wl.s * wl.d * esz))
+    per_step = max(1, min(len(rows), threads, cap, args.ref_rows or len(rows)))
+    data = [src.row(b, g) for (b, g) in rows[:per_step]]
+    used = min(threads, per_step)
+
+    def one_step(ex):
+        list(ex.map(lambda r: oracle_row(wl, r), data))
+
+    with cf.ThreadPoolExecutor(max_workers=used) as ex:
+        for _ in range(args.warmup):
+            one_step(ex)
         t0 = time.perf_counter()
-        oracle_sample(wl, host, float("inf"), max_rows=rows_per_step)
-        t_total += time.perf_counter() - t0
-    frac = rows_per_step / (wl.b * wl.hkv)
+        for _ in range(args.steps):
+            one_step(ex)
+        t_total = time.perf_counter() - t0
+    frac = per_step / len(rows)
     value = wl.b * frac * args.steps / t_total
-    sample = f"{rows_per_step} of {wl.b * wl.hkv} (batch, kv-head) rows per step"
+    sample = (f"{per_step} of {len(rows)} (batch, kv-head) rows per step (label build + scores + top-k + "
+              f"attention), one per thread")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {**workload_config(wl, None), "l2": "not applicable (CPU oracle)"},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle", "sample": sample,
+                             "cpu_model": cpu_model()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
 
@@ -601,17 +713,27 @@ def workload_config(wl, plan):
 
 # ------------------------------------------------------------------ main
 
+DEFAULT_CONFIG = 2          # the largest single-GPU workload is the headline
+DEFAULT_ALSO = (1, 3, 4)    # nested records
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", type=int, default=1, help="workload index (0-4)")
-    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time for cpu_baseline")
-    ap.add_argument("--ref-rows", type=int, default=8, help="rows per reference-arm step")
+    ap.add_argument("--config", type=int, default=None,
+                    help=f"headline workload index (0-4; default {DEFAULT_CONFIG})")
+    ap.add_argument("--also", default=None,
+                    help="comma-separated workload indices measured after the headline and nested under "
+                         "'configs' (default: the other full-size workloads; '' for none)")
+    ap.add_argument("--cpu-budget", type=float, default=8.0,
+                    help="seconds of oracle time per cpu_baseline leg (headline; nested records use half)")
+    ap.add_argument("--ref-rows", type=int, default=0,
+                    help="rows per reference-arm step (0: one per host thread)")
     ap.add_argument("--label", default=None, choices=["f32", "bf16", "int4"],
-                    help="override the workload's label cache dtype (measurement variants)")
+                    help="override the headline workload's label cache dtype (measurement variants)")
     ap.add_argument("--offload", action="store_true",
                     help="also time the step with the K/V caches in pinned host memory")
     ap.add_argument("--timing", default="rotate", choices=["rotate", "flush"],
@@ -620,7 +742,12 @@ def main():
     ap.add_argument("--flush", default="write_read", choices=["write_read", "copy", "fill"],
                     help="L2 eviction between timed steps: fill then read (default), D2D copy, or fill kernel")
     args = ap.parse_args()
-    wl = synth.workload(args.config)
+    head = DEFAULT_CONFIG if args.config is None else args.config
+    if args.also is None:
+        also = [i for i in DEFAULT_ALSO if i != head] if args.config is None else []
+    else:
+        also = [int(x) for x in args.also.split(",") if x.strip()]
+    wl = synth.workload(head)
     if args.label and args.label != wl.label_dtype:
         if args.label != "int4" and args.label != wl.kv_dtype:
             raise SystemExit("an fp label cache has the key cache's dtype")
@@ -642,16 +769,32 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
     try:
         r = run_ours(args, wl, rank, local_rank, world)
-        line = None
-        if rank == 0:
-            line = report(args, wl, r, world)
+        line = report(args, wl, r, world, head, args.cpu_budget) if rank == 0 else None
+        del r
+        torch.cuda.empty_cache()
+        nested = {}
+        for i in also:
+            wl_i = synth.workload(i)
+            r_i = run_ours(args, wl_i, rank, local_rank, world)
+            if rank == 0:
+                rec = report(args, wl_i, r_i, world, i, args.cpu_budget / 2)
+                nested[wl_i.name] = {k: rec[k] for k in NESTED_KEYS if k in rec}
+            del r_i
+            torch.cuda.empty_cache()
         barrier()
         if line:
+            if nested:
+                line["configs"] = nested
             print(json.dumps(line))
     finally:
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()
+
+
+NESTED_KEYS = ("value", "unit", "ms_per_step", "steps", "config", "hbm_gbs", "roofline", "step_us",
+               "cpu_baseline", "e2e", "gpu_launches", "clocks", "dense_baseline", "prefill_label_build",
+               "offload")
 
 
 def l2_note(args, r) -> str:
@@ -665,19 +808,13 @@ def l2_note(args, r) -> str:
                if args.flush == "write_read" else ""))
 
 
-def report(args, wl, r, world):
+def report(args, wl, r, world, index, cpu_budget):
     ab = algorithmic_bytes(wl, r["out_esz"])
     peaks = measured_peaks()
     value = job_value(wl.b, world, args.steps, r["max_s"])
     dec_avg_s = sum(r["step_ms"]) / len(r["step_ms"]) / 1e3  # the step is one launch of the kernel
     achieved = ab["total"] / dec_avg_s / 1e9
-    cpu = None
-    if world == 1:
-        host = host_arrays(wl, r["host"])
-        t_step, rows = oracle_sample(wl, host, args.cpu_budget)
-        cpu = {"value": wl.b / t_step, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": f"{rows} of {wl.b * wl.hkv} (batch, kv-head) rows of one step "
-                         f"(label build + scores + top-k + attention), scaled to the full step"}
+    cpu = cpu_baseline(wl, r["rows"], cpu_budget) if world == 1 else None
     dense_s = r["dense_ms"] / 1e3
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -690,8 +827,9 @@ def report(args, wl, r, world):
         "pct_of_measured_hbm": 100 * achieved / peaks["hbm_gbs"],
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"],
-                     "traffic": (recorded_traffic(args.config)
-                                 if wl.label_dtype == synth.workload(args.config).label_dtype else None), "kernel": "ds_decode_kernel",
+                     "traffic": (recorded_traffic(index)
+                                 if wl.label_dtype == synth.workload(index).label_dtype else None),
+                     "kernel": "ds_decode_kernel",
                      "algorithmic_bytes_per_launch": ab["total"], "avg_launch_us": dec_avg_s * 1e6},
         "step_us": dec_avg_s * 1e6,
         "cpu_baseline": cpu,
@@ -706,8 +844,9 @@ def report(args, wl, r, world):
                            / 1e3 / dec_avg_s,
                            "byte_ratio": ab["dense_total"] / ab["total"],
                            "dense_hbm_gbs": ab["dense_total"] / dense_s / 1e9},
-        "prefill_label_build": {"us": r["prefill_ms"] * 1e3,
-                                "gbs": prefill_bytes(wl) / (r["prefill_ms"] / 1e3) / 1e9},
+        "prefill_label_build": {"us": r["prefill_ms"] * 1e3, "bytes": prefill_bytes(wl),
+                                "gbs": prefill_bytes(wl) / (r["prefill_ms"] / 1e3) / 1e9,
+                                "frac": prefill_bytes(wl) / (r["prefill_ms"] / 1e3) / 1e9 / peaks["hbm_gbs"]},
         "wall_s_timed_region": r["wall_s"],
     }
     if r["offload"]:

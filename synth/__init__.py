@@ -194,6 +194,21 @@ def new_token(wl: Workload, step: int = 0):
             to_storage(qn, wl.kv_dtype))
 
 
+def decode_row_inputs(wl: Workload, b: int, g: int, seed_offset: int = 0):
+    """The query heads of kv head g ([1, G, D]) and that head's K and V
+    ([1, 1, S, D]) for batch entry b, drawn on the host with the recipe of
+    :func:`decode_inputs` (N(0, 1), the planted channels scaled in K and q)
+    from a seed of their own: one row of a workload too large to draw whole."""
+    chans = outlier_channels(wl)[g:g + 1]
+    base = 1000 * wl.index + 100 * seed_offset + 10_000_000 + 4 * (b * wl.hkv + g)
+    q = normal((1, wl.g, wl.d), base + 0)
+    q[:, :, chans[0]] *= np.float32(wl.outlier_scale)
+    k = normal((1, 1, wl.s, wl.d), base + 1)
+    v = normal((1, 1, wl.s, wl.d), base + 2)
+    _plant_kv(k, chans, wl.outlier_scale)
+    return to_storage(q, wl.kv_dtype), to_storage(k, wl.kv_dtype), to_storage(v, wl.kv_dtype)
+
+
 @dataclass
 class CalibInputs:
     wl: Workload
