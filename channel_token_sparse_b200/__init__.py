@@ -21,7 +21,7 @@ import os
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libds.so")
 
-DS_OK, DS_ERR_INVALID_ARG, DS_ERR_UNSUPPORTED, DS_ERR_CUDA, DS_ERR_WORKSPACE = range(5)
+DS_OK, DS_ERR_INVALID_ARG, DS_ERR_UNSUPPORTED, DS_ERR_CUDA, DS_ERR_WORKSPACE, DS_ERR_TIMEOUT = range(6)
 DS_F32, DS_BF16, DS_F16, DS_INT4 = range(4)
 DS_FALLBACK_PER_ENTRY, DS_FALLBACK_BATCH = range(2)
 DS_CRIT_LEANK_RATIO, DS_CRIT_Q_OUTLIER, DS_CRIT_K_OUTLIER, DS_CRIT_QK_OUTLIER, DS_CRIT_QK_CHUNKED = range(5)
@@ -53,6 +53,9 @@ SIGNATURES = {
     "ds_sparse_decode_plan": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, _i, C.POINTER(_i), C.POINTER(_i),
                                    C.POINTER(_i)]),
     "ds_sparse_decode_set_cluster": (None, [_i]),
+    "ds_sparse_decode_tune": (_i, [C.c_char_p, _i]),
+    "ds_check_device": (_i, [_vp]),
+    "ds_selftest_bounded_wait": (_i, [_i, _vp]),
     "ds_sparse_decode_workspace": (_i, [_i, _i, _i, _i, _i, _i, _i, C.POINTER(_sz)]),
     "ds_dense_decode": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _i, _vp]),
 }
@@ -110,19 +113,32 @@ def _ptr(t):
     return None if t is None else C.c_void_p(t.data_ptr())
 
 
+_mapped = {}  # host address of a pinned tensor -> its device-mapped address
+
+
 def _ptr_kv(t):
-    """Device address of a key/value cache: a CUDA tensor, or a pinned host
-    tensor mapped into the device's address space (DS-Offload: the kernels
-    then read the rows they need over the host link)."""
+    """Device address of a tensor the kernels may read (or write) over the
+    host link: a CUDA tensor, or a pinned host tensor mapped into the
+    device's address space (DS-Offload keeps K/V there; a decode step may also
+    take its new rows and query from there and write its output there)."""
+    if t is None:
+        return None
     if t.is_cuda:
         return C.c_void_p(t.data_ptr())
     if not t.is_pinned():
-        raise ValueError("a key/value cache in host memory must be pinned")
-    from cuda.bindings import runtime as rt
-    err, dptr = rt.cudaHostGetDevicePointer(t.data_ptr(), 0)
-    if err != rt.cudaError_t.cudaSuccess:
-        raise ValueError(f"pinned host cache is not mapped for the device: {err}")
-    return C.c_void_p(int(dptr))
+        raise ValueError("a tensor in host memory must be pinned")
+    hp = t.data_ptr()
+    dp = _mapped.get(hp)
+    if dp is None:
+        from cuda.bindings import runtime as rt
+        err, dp = rt.cudaHostGetDevicePointer(hp, 0)
+        if err != rt.cudaError_t.cudaSuccess:
+            raise ValueError(f"pinned host tensor is not mapped for the device: {err}")
+        dp = int(dp)
+        if len(_mapped) > 4096:
+            _mapped.clear()
+        _mapped[hp] = dp
+    return C.c_void_p(dp)
 
 
 def _need_cuda_or_pinned(*ts):
@@ -159,6 +175,18 @@ def _need_cuda(*ts):
 def set_cluster(n: int) -> None:
     """Force CTAs per (b, kv head) cluster (1..16, power of two); 0 = automatic."""
     lib().ds_sparse_decode_set_cluster(int(n))
+
+
+def check_device(stream=None) -> None:
+    """Raise DSError(DS_ERR_TIMEOUT) if a kernel gave up a bounded wait since
+    the last check (synchronises the stream)."""
+    _check(lib().ds_check_device(_stream(stream)))
+
+
+def tune(name: str, value: int) -> None:
+    """Set a decode tuning knob ("stagger", "att_prefetch", "scan_prefetch");
+    a negative value restores its default."""
+    _check(lib().ds_sparse_decode_tune(name.encode(), int(value)))
 
 
 def plan(b, hq, hkv, s, d, c, topk, kv_dtype=DS_BF16, label_dtype=DS_BF16):
@@ -326,10 +354,14 @@ def decode_step_kv(q, k_new, v_new, k, v, label, idx, s: int, topk: int, lscale=
                    out_dtype=None, sm_scale: float = 0.0, sel_out=None, score_out=None, stream=None):
     """decode_step that first writes the new token's rows k_new, v_new
     [B, Hkv, D] into k, v at position s - 1 (in the same launch); returns
-    out [B, Hq, D]."""
+    out [B, Hq, D]. q, k_new, v_new and out may be pinned host tensors: the
+    kernel then reads the step's inputs and writes its output over the host
+    link itself, so a step from host buffers is this one call."""
     torch = _torch()
-    _need_cuda_or_pinned(k, v)
-    _need_cuda(q, k_new, v_new, label, idx, lscale, lzero, out, sel_out, score_out)
+    _need_cuda_or_pinned(k, v, q, k_new, v_new)
+    if out is not None:
+        _need_cuda_or_pinned(out)
+    _need_cuda(label, idx, lscale, lzero, sel_out, score_out)
     b, hq, d = q.shape
     _, hkv, s_cap, _ = k.shape
     c = idx.shape[1]
@@ -337,12 +369,12 @@ def decode_step_kv(q, k_new, v_new, k, v, label, idx, s: int, topk: int, lscale=
     if k_new.dtype != k.dtype or v_new.dtype != v.dtype:
         raise TypeError("k_new / v_new must have the caches' dtype")
     if out is None:
-        out = torch.empty((b, hq, d), dtype=out_dtype or torch.float32, device=q.device)
+        out = torch.empty((b, hq, d), dtype=out_dtype or torch.float32, device=label.device)
     odt = DS_F32 if out.dtype == torch.float32 else DS_BF16
-    _check(lib().ds_decode_step_kv(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr_kv(k), _ptr_kv(v), kdt, _ptr(label),
-                                   _label_args(label, lscale, lzero, kdt), _ptr(lscale), _ptr(lzero),
+    _check(lib().ds_decode_step_kv(_ptr_kv(q), _ptr_kv(k_new), _ptr_kv(v_new), _ptr_kv(k), _ptr_kv(v), kdt,
+                                   _ptr(label), _label_args(label, lscale, lzero, kdt), _ptr(lscale), _ptr(lzero),
                                    _ptr(idx), b, hq, hkv, s, s_cap, d, c, topk, float(sm_scale),
-                                   _ptr(out), odt, _ptr(sel_out), _ptr(score_out), _stream(stream)))
+                                   _ptr_kv(out), odt, _ptr(sel_out), _ptr(score_out), _stream(stream)))
     return out
 
 

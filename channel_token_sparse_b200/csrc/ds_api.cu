@@ -6,6 +6,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <string>
 #include <unordered_map>
 
 #include "ds.h"
@@ -16,6 +17,25 @@ namespace {
 
 thread_local char g_err[256] = "";
 std::atomic<int> g_cluster_override{0};
+// Tuning knobs (ds_sparse_decode_tune)
+std::atomic<int> g_stagger_pct{100};  // share of the first group a held-back CTA waits for (0: off)
+std::atomic<int> g_att_prefetch{4};   // attention: tiles prefetched into L2 ahead of the copy ring
+std::atomic<int> g_scan_prefetch{2};  // label scan without the ring: rounds prefetched into L2 ahead
+
+// Small device words of the library: [0], [1] the counters of the decode
+// kernel's staggered first wave (see DecodeParams; the kernel's last CTA
+// resets them, so every launch finds them at zero; concurrent decode launches
+// on one device share them, which can only delay a held-back CTA up to its
+// poll limit, never change a result); [2] the status word in which a kernel
+// records a bounded wait that gave up (bit = where; read and cleared by
+// ds_check_device).
+static __device__ __align__(16) unsigned int g_decode_sched[4];
+constexpr int kStatusWord = 2;
+
+std::mutex g_sched_mu;
+struct SchedAddr { unsigned long long ctx; unsigned int* ptr; };
+SchedAddr g_sched_addr[16];
+int g_sched_used = 0, g_sched_next = 0;
 
 ds_status fail(ds_status st, const char* fmt, ...) {
     va_list ap;
@@ -182,6 +202,96 @@ ds_status launch_decode(ds::DecodeKernel kern, const ds::DecodeParams& p, int ro
     return DS_OK;
 }
 
+}  // namespace
+
+namespace ds {
+
+// Process-unique id of the calling thread's current CUDA context (0 and
+// false when there is none or the driver does not provide one). Caches of
+// device addresses are keyed by it: a context created after a device reset
+// gets a new id, and its modules (and their __device__ variables) may sit
+// elsewhere. The driver functions are fetched through the runtime, so the
+// library does not link the driver library itself.
+bool current_context_id(unsigned long long* id) {
+    using GetCurrent = int (*)(void**);
+    using GetId = int (*)(void*, unsigned long long*);
+    static GetCurrent get_current = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            f = nullptr;
+        return reinterpret_cast<GetCurrent>(f);
+    }();
+    static GetId get_id = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &f, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            f = nullptr;
+        return reinterpret_cast<GetId>(f);
+    }();
+    void* ctx = nullptr;
+    *id = 0;
+    return get_current && get_id && get_current(&ctx) == 0 && ctx && get_id(ctx, id) == 0;
+}
+
+}  // namespace ds
+
+namespace {
+
+// A barrier that nothing completes: the bounded wait runs out after
+// `limit_ns` and records site bit 0 (ds_selftest_bounded_wait).
+__global__ void ds_selftest_wait_kernel(unsigned int* err, unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        ds::mbar_init(&bar, 1);
+        ds::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) ds::mbar_wait_bounded(&bar, 0, err, 0, limit_ns);
+}
+
+// Device address of g_decode_sched in the current context, cached per
+// context (host code only has the array's name as a host-side stand-in).
+cudaError_t sched_counters(unsigned int** out) {
+    unsigned long long ctx = 0;
+    const bool keyed = ds::current_context_id(&ctx);
+    std::lock_guard<std::mutex> lk(g_sched_mu);
+    if (keyed)
+        for (int i = 0; i < g_sched_used; ++i)
+            if (g_sched_addr[i].ctx == ctx) { *out = g_sched_addr[i].ptr; return cudaSuccess; }
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_sched);
+    if (e != cudaSuccess) return e;
+    if (keyed || ds::current_context_id(&ctx)) {
+        g_sched_addr[g_sched_next] = SchedAddr{ctx, static_cast<unsigned int*>(p)};
+        g_sched_next = (g_sched_next + 1) % 16;
+        if (g_sched_used < 16) ++g_sched_used;
+    }
+    *out = static_cast<unsigned int*>(p);
+    return cudaSuccess;
+}
+
+// Staggered first wave: of the CTAs resident at once, the first half (whole
+// clusters) streams its label rows at once, the second half waits for it
+// (see DecodeParams). Rows that only fill part of a wave, or fewer than two
+// clusters, are not staggered.
+ds_status plan_stagger(ds::DecodeParams& p, int rows, int N, int slots) {
+    p.sched = nullptr;
+    const int pct = g_stagger_pct.load();
+    const int grid = rows * N;
+    const int wave = (grid < slots ? grid : slots) / N * N;
+    if (pct <= 0 || wave < 2 * N) return DS_OK;
+    cudaError_t e = sched_counters(&p.sched);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+    p.stagger_a = wave / 2 / N * N;
+    p.stagger_end = wave;
+    p.stagger_target = (p.stagger_a * pct + 99) / 100;
+    p.stagger_polls = 400;  // ~40-80 us of __nanosleep(100) at most
+    return DS_OK;
+}
+
 ds_status check_common(int b, int hq, int hkv, int s, int s_cap, int d, ds_dtype kvdt) {
     if (b < 1 || hkv < 1 || hq < 1) return fail(DS_ERR_INVALID_ARG, "b, hq and hkv must be >= 1");
     if (hq % hkv) return fail(DS_ERR_INVALID_ARG, "hq (%d) must be a multiple of hkv (%d)", hq, hkv);
@@ -249,6 +359,13 @@ ds_status run_label(const void* k, ds_dtype kdt, const int32_t* idx, int b, int 
     if (!aligned16(k) || !aligned16(idx)) return fail(DS_ERR_INVALID_ARG, "k/idx not 16-byte aligned");
     ds::LabelArgs a{k, kdt == DS_BF16, label_dt == DS_INT4, idx, b, hkv, t_begin, t_end, s_cap, d, c,
                     label, lscale, lzero};
+    unsigned int* words = nullptr;
+    if (!pg && t_end - t_begin > 1) {
+        cudaError_t e = sched_counters(&words);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+        a.err = words + kStatusWord;
+        a.sms = sm_count();
+    }
     if (pg) {
         a.block_table = pg->bt;
         a.max_blocks = pg->max_blocks;
@@ -271,6 +388,7 @@ const char* ds_status_string(ds_status st) {
     case DS_ERR_UNSUPPORTED: return "DS_ERR_UNSUPPORTED";
     case DS_ERR_CUDA: return "DS_ERR_CUDA";
     case DS_ERR_WORKSPACE: return "DS_ERR_WORKSPACE";
+    case DS_ERR_TIMEOUT: return "DS_ERR_TIMEOUT";
     }
     return "DS_ERR_UNKNOWN";
 }
@@ -278,6 +396,52 @@ const char* ds_status_string(ds_status st) {
 const char* ds_last_error(void) { return g_err; }
 
 void ds_sparse_decode_set_cluster(int n) { g_cluster_override.store(n); }
+
+ds_status ds_sparse_decode_tune(const char* name, int value) {
+    if (!name) return fail(DS_ERR_INVALID_ARG, "name is NULL");
+    const std::string n(name);
+    if (n == "stagger") {
+        if (value > 100) return fail(DS_ERR_INVALID_ARG, "stagger is a percentage (0..100, <0 default)");
+        g_stagger_pct.store(value < 0 ? 100 : value);
+    } else if (n == "att_prefetch") {
+        if (value > 16) return fail(DS_ERR_INVALID_ARG, "att_prefetch: 0..16 tiles (<0 default)");
+        g_att_prefetch.store(value < 0 ? 4 : value);
+    } else if (n == "scan_prefetch") {
+        if (value > 8) return fail(DS_ERR_INVALID_ARG, "scan_prefetch: 0..8 rounds (<0 default)");
+        g_scan_prefetch.store(value < 0 ? 2 : value);
+    } else {
+        return fail(DS_ERR_INVALID_ARG, "unknown tuning knob '%s'", name);
+    }
+    return DS_OK;
+}
+
+ds_status ds_selftest_bounded_wait(int polls, cudaStream_t stream) {
+    if (polls < 1 || polls > 1000000) return fail(DS_ERR_INVALID_ARG, "polls must be in [1, 1000000]");
+    unsigned int* words = nullptr;
+    cudaError_t e = sched_counters(&words);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+    ds_selftest_wait_kernel<<<1, 32, 0, stream>>>(words + kStatusWord, (unsigned long long)polls * 1000ull);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+    return DS_OK;
+}
+
+ds_status ds_check_device(cudaStream_t stream) {
+    unsigned int* words = nullptr;
+    cudaError_t e = sched_counters(&words);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+    unsigned int w = 0;
+    e = cudaMemcpyAsync(&w, words + kStatusWord, sizeof w, cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device status");
+    if (!w) return DS_OK;
+    const unsigned int zero = 0;
+    e = cudaMemcpyAsync(words + kStatusWord, &zero, sizeof zero, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device status");
+    return fail(DS_ERR_TIMEOUT, "a kernel gave up a bounded wait (sites 0x%x: bit 0 self-test, "
+                "bit 1 label build stage, bit 2 decode stage)", w);
+}
 
 ds_status ds_calibrate_workspace_size(int n_samples, int hq, int hkv, int w, int s, int d,
                                       size_t* bytes) {
@@ -465,6 +629,9 @@ ds_status sparse_decode_impl(const void* q, const void* k, const void* v, ds_dty
     p.qscale = scale * 1.4426950408889634f;
     p.out_bf16 = out_dt == DS_BF16;
     p.dense = 0;
+    if ((r = plan_stagger(p, rows, pl.N, kCtasPerSm * sm_count())) != DS_OK) return r;
+    p.att_prefetch = g_att_prefetch.load();
+    p.scan_prefetch = g_scan_prefetch.load();
     return launch_decode(kern, p, rows, pl, stream);
 }
 

@@ -211,9 +211,8 @@ cudaError_t launch_calib(const CalibArgs& a, cudaStream_t st) {
 // ------------------------------------------------ calibration without allocation
 //
 // For callers that cannot obtain device memory from cudaMalloc or a caching
-// allocator: code running while a CUDA graph is being captured, hosts that
-// hand a plugin only fixed tensors and own every allocation, or runtimes with
-// a preallocated device budget. The scratch then lives in this fixed
+// allocator: hosts that hand a plugin only fixed tensors and own every
+// allocation, or runtimes with a preallocated device budget. The scratch then lives in this fixed
 // file-scope array, which every GPU that loads the library keeps until exit.
 // All calls share it and each call first clears the part it uses; calls that
 // overlap on the GPU (different streams, no ordering between them) race on it.
@@ -223,24 +222,32 @@ constexpr size_t kStaticCalibDoubles = 131072;  // 1 MiB
 static __device__ __align__(256) double g_calib_static_scratch[kStaticCalibDoubles];
 
 std::mutex g_static_mu;
-void* g_static_ptr[64] = {};  // device address of the array, per device ordinal
+struct StaticAddr { unsigned long long ctx; void* ptr; };
+StaticAddr g_static_addr[16];  // most recent contexts first-come
+int g_static_used = 0, g_static_next = 0;
 
-// Device address of the scratch array on the current device. Host code sees
-// the array's name as a host-side stand-in, so the address is looked up once
-// per device (with that device current) and cached.
+// Device address of the scratch array in the current context. Host code sees
+// the array's name as a host-side stand-in, not a device address, so the
+// address is asked of the runtime with the device current and cached per
+// context (keyed by the context's process-unique id: after a device reset the
+// new context's copy of the array is looked up afresh).
 cudaError_t static_scratch(void** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    unsigned long long ctx = 0;
+    const bool keyed = ds::current_context_id(&ctx);
     std::lock_guard<std::mutex> lk(g_static_mu);
-    if (!g_static_ptr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_calib_static_scratch);
-        if (e != cudaSuccess) return e;
-        g_static_ptr[dev] = p;
+    if (keyed)
+        for (int i = 0; i < g_static_used; ++i)
+            if (g_static_addr[i].ctx == ctx) { *out = g_static_addr[i].ptr; return cudaSuccess; }
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_calib_static_scratch);
+    if (e != cudaSuccess) return e;
+    // the lookup makes the device's primary context current when none was
+    if (keyed || ds::current_context_id(&ctx)) {
+        g_static_addr[g_static_next] = StaticAddr{ctx, p};
+        g_static_next = (g_static_next + 1) % 16;
+        if (g_static_used < 16) ++g_static_used;
     }
-    *out = g_static_ptr[dev];
+    *out = p;
     return cudaSuccess;
 }
 

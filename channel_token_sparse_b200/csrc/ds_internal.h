@@ -21,6 +21,10 @@ DecodeKernel decode_kernel_f32_i4_paged(int D, int C, int GT);
 DecodeKernel decode_kernel_bf16_fp_paged(int D, int C, int GT);
 DecodeKernel decode_kernel_bf16_i4_paged(int D, int C, int GT);
 
+// Process-unique id of the current CUDA context (false if there is none):
+// the key of the per-context caches of __device__ variable addresses.
+bool current_context_id(unsigned long long* id);
+
 struct LabelArgs {
     const void* k;
     bool kdt_bf16;
@@ -32,6 +36,8 @@ struct LabelArgs {
     uint16_t* lzero;
     const int32_t* block_table = nullptr;  // paged key cache (see ds_label.cu)
     int max_blocks = 0, page_shift = 0, num_blocks = 0;
+    unsigned int* err = nullptr;  // device word recording a bounded wait that gave up (pipelined build)
+    int sms = 148;                // SMs of the device (pipelined build grid)
 };
 cudaError_t launch_label(const LabelArgs& a, cudaStream_t st);
 

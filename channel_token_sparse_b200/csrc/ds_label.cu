@@ -70,9 +70,157 @@ __global__ void __launch_bounds__(kLabNT) ds_label_kernel(const TKV* __restrict_
     }
 }
 
+// Dense key cache, many tokens (prefill): persistent CTAs stream blocks of
+// consecutive key rows -- one contiguous span of kBulkStage bytes per
+// (row, block) item -- through a kBulkStages-deep shared-memory ring with 1-D
+// bulk copies (thread 0 issues them; an mbarrier per stage counts the bytes
+// in), so the next blocks' reads are in flight while the current one is
+// gathered or packed. Same results as ds_label_kernel.
+constexpr int kBulkStage = 16384;  // bytes of key rows per stage
+constexpr int kBulkStages = 4;
+constexpr int kBulkNT = 256;
+// packing threads per token (4-bit): each takes c / kPackLanes channels
+constexpr int kPackLanes = 4;
+
+__host__ __device__ constexpr int bulk_smem_bytes() { return kBulkStages * kBulkStage + kBulkStages * 8; }
+
+template <typename TKV, int LK, int D>
+__global__ void __launch_bounds__(kBulkNT, 2) ds_label_bulk_kernel(const TKV* __restrict__ k,
+                                                                  const int32_t* __restrict__ idx, int hkv,
+                                                                  int t_begin, int t_end, int s_cap, int c,
+                                                                  int rows, uint8_t* __restrict__ label,
+                                                                  uint16_t* __restrict__ lscale,
+                                                                  uint16_t* __restrict__ lzero,
+                                                                  unsigned int* __restrict__ err) {
+    using E = Elem<TKV>;
+    constexpr int kRowBytes = D * E::kBytes;
+    constexpr int kTok = kBulkStage / kRowBytes;  // tokens per stage
+    extern __shared__ __align__(128) uint8_t sm[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + kBulkStages * kBulkStage);
+    const int tid = threadIdx.x;
+    const int nblk = (t_end - t_begin + kTok - 1) / kTok;  // blocks per row
+    const long long items = (long long)rows * nblk;
+    if (tid == 0) {
+        for (int i = 0; i < kBulkStages; ++i) mbar_init(&full[i], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    auto issue = [&](long long it, int slot) {
+        const int row = (int)(it / nblk), blk = (int)(it - (long long)row * nblk);
+        const int tb = t_begin + blk * kTok;
+        const int nt = min(kTok, t_end - tb);
+        const uint32_t bytes = (uint32_t)(nt * kRowBytes);
+        mbar_arrive_expect_tx(&full[slot], bytes);
+        bulk_g2s(sm + slot * kBulkStage, k + ((size_t)row * s_cap + tb) * D, bytes, &full[slot]);
+    };
+    if (tid == 0)
+        for (int i = 0; i < kBulkStages; ++i) {
+            const long long it = blockIdx.x + (long long)i * gridDim.x;
+            if (it < items) issue(it, i);
+        }
+    int g_cur = -1;
+    int my_idx[128 / kPackLanes > 1 ? 128 / kPackLanes : 1];  // 4-bit: this thread's channels
+    int fp_idx = 0;                                            // fp: this thread's channel (tid % c)
+    int j = 0;
+    for (long long it = blockIdx.x; it < items; it += gridDim.x, ++j) {
+        const int slot = j % kBulkStages;
+        const int row = (int)(it / nblk), blk = (int)(it - (long long)row * nblk);
+        const int g = row % hkv;
+        const int tb = t_begin + blk * kTok;
+        const int nt = min(kTok, t_end - tb);
+        const size_t tok0 = (size_t)row * s_cap + tb;
+        if (g != g_cur) {
+            g_cur = g;
+            if constexpr (LK == 0) {
+                fp_idx = min(max(__ldg(idx + (size_t)g * c + tid % c), 0), D - 1);
+            } else {
+                const int per = c / kPackLanes, q = tid % kPackLanes;
+                for (int e = 0; e < per; ++e) my_idx[e] = min(max(__ldg(idx + (size_t)g * c + q * per + e), 0), D - 1);
+            }
+        }
+        const bool ok = mbar_wait_bounded(&full[slot], (uint32_t)((j / kBulkStages) & 1), err, 1);
+        const TKV* rows_s = reinterpret_cast<const TKV*>(sm + slot * kBulkStage);
+        if (ok) {
+            if constexpr (LK == 0) {
+                // thread tid always handles channel tid % c (c divides the CTA size)
+                TKV* out = reinterpret_cast<TKV*>(label) + tok0 * c;
+                for (int e = tid; e < nt * c; e += kBulkNT) out[e] = rows_s[(e / c) * D + fp_idx];
+            } else {
+                // kPackLanes threads per token, c / kPackLanes channels each:
+                // the arithmetic of pack_int4_row, with mn / mx combined over
+                // the lanes (fminf / fmaxf do not depend on the order)
+                const int per = c / kPackLanes, q = tid % kPackLanes;
+                for (int t = tid / kPackLanes; t < ((nt + 7) & ~7); t += kBulkNT / kPackLanes) {
+                    const bool live = t < nt;
+                    const TKV* x = rows_s + (size_t)(live ? t : 0) * D;
+                    float mn = E::to_f32(x[my_idx[0]]), mx = mn;
+                    for (int e = 1; e < per; ++e) {
+                        const float v = E::to_f32(x[my_idx[e]]);
+                        mn = fminf(mn, v);
+                        mx = fmaxf(mx, v);
+                    }
+#pragma unroll
+                    for (int o = 1; o < kPackLanes; o <<= 1) {
+                        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                    }
+                    const float step = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+                    const uint16_t sh = __half_as_ushort(__float2half_rn(step));
+                    const uint16_t zh = __half_as_ushort(__float2half_rn(mn));
+                    const float sc = fp16_bits_to_f32(sh), z = fp16_bits_to_f32(zh);
+                    if (live) {
+                        uint8_t* dst = label + (tok0 + t) * (size_t)(c / 2) + q * per / 2;
+                        for (int e = 0; e < per; e += 2) {
+                            uint32_t nib[2];
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                uint32_t code = 0;
+                                if (sc > 0.f) {
+                                    float qv = rintf(__fdiv_rn(__fsub_rn(E::to_f32(x[my_idx[e + h]]), z), sc));
+                                    qv = fminf(fmaxf(qv, 0.f), 15.f);
+                                    code = (uint32_t)qv;
+                                }
+                                nib[h] = code;
+                            }
+                            dst[e / 2] = (uint8_t)(nib[0] | (nib[1] << 4));
+                        }
+                        if (q == 0) {
+                            lscale[tok0 + t] = sh;
+                            lzero[tok0 + t] = zh;
+                        }
+                    }
+                }
+            }
+        }
+        __syncthreads();  // every thread is done with the slot
+        if (!__syncthreads_and(ok)) break;  // a copy never arrived: leave (recorded in *err)
+        if (tid == 0) {
+            const long long nx = it + (long long)kBulkStages * gridDim.x;
+            if (nx < items) issue(nx, slot);
+        }
+    }
+}
+
 template <typename TKV, int LK, int D>
 static cudaError_t launch_label_t(const LabelArgs& a, cudaStream_t st) {
     const int n = a.t_end - a.t_begin;
+    constexpr int kTok = kBulkStage / (D * Elem<TKV>::kBytes);
+    const long long items = (long long)a.b * a.hkv * ((n + kTok - 1) / kTok);
+    if (!a.block_table && a.err && items >= 2 * (long long)a.sms && (LK == 0 || a.c >= 2 * kPackLanes)) {
+        static bool attr = false;  // set once per process (the attribute is per function)
+        if (!attr) {
+            const cudaError_t e = cudaFuncSetAttribute(ds_label_bulk_kernel<TKV, LK, D>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       bulk_smem_bytes());
+            if (e != cudaSuccess) return e;
+            attr = true;
+        }
+        const long long grid = items < 2LL * a.sms ? items : 2LL * a.sms;
+        ds_label_bulk_kernel<TKV, LK, D><<<(unsigned)grid, kBulkNT, bulk_smem_bytes(), st>>>(
+            reinterpret_cast<const TKV*>(a.k), a.idx, a.hkv, a.t_begin, a.t_end, a.s_cap, a.c, a.b * a.hkv,
+            reinterpret_cast<uint8_t*>(a.label), a.lscale, a.lzero, a.err);
+        return cudaGetLastError();
+    }
     dim3 grid((n + kTokens - 1) / kTokens, a.b * a.hkv);
     ds_label_kernel<TKV, LK, D><<<grid, kLabNT, 0, st>>>(
         reinterpret_cast<const TKV*>(a.k), a.idx, a.hkv, a.t_begin, a.t_end, a.s_cap, a.c,

@@ -62,7 +62,8 @@ typedef enum {
     DS_ERR_INVALID_ARG = 1,
     DS_ERR_UNSUPPORTED = 2,
     DS_ERR_CUDA = 3,
-    DS_ERR_WORKSPACE = 4
+    DS_ERR_WORKSPACE = 4,
+    DS_ERR_TIMEOUT = 5
 } ds_status;
 
 typedef enum { DS_F32 = 0, DS_BF16 = 1, DS_F16 = 2, DS_INT4 = 3 } ds_dtype;
@@ -132,18 +133,22 @@ DS_API ds_status ds_calibrate_channels_criterion(const void* q_win, const void* 
                                                  int chunk, float* score_out, int32_t* idx_out,
                                                  void* ws, size_t ws_bytes, cudaStream_t stream);
 
-/* Calibration for callers that cannot allocate device memory -- code that
- * runs while a CUDA graph is being captured, plugins whose host framework owns
- * every allocation, or runtimes with a fixed device budget. It has no
+/* Calibration for callers that cannot allocate device memory: plugins whose
+ * host framework owns every allocation and hands them only fixed tensors, or
+ * runtimes that work inside a device budget fixed up front, so that a call
+ * to cudaMalloc (or to an allocator that may call it) is not open to them.
+ * It has no
  * counterpart on the pages; it computes exactly what ds_calibrate_channels
  * computes, with the same arguments minus the workspace. Its scratch is a
  * fixed 1 MiB device array inside the library (held by every GPU that loads
  * the library until the process exits), so it needs
  * n_samples * hkv * (2*d + 1) * 8 <= 1048576 bytes (ds_calibrate_workspace_size
  * gives the figure); larger problems get DS_ERR_WORKSPACE with the numbers.
- * It allocates nothing and calls no allocating routine. The first call on a
- * device looks up the array's device address (once per device, with that
- * device current); make that first call before any stream capture. All calls
+ * It allocates nothing and calls no allocating routine. The first call in a
+ * CUDA context looks up the array's device address (with that device current)
+ * and caches it for the context; a context created later, e.g. after a device
+ * reset, is looked up afresh on its first call. Make that first call before
+ * any stream capture. All calls
  * share the array and each clears the part it uses: calls that may run
  * concurrently on the GPU (different streams without ordering) race on it. */
 DS_API ds_status ds_calibrate_channels_noalloc(const void* q_win, const void* k, ds_dtype dt,
@@ -315,6 +320,41 @@ DS_API ds_status ds_sparse_decode_plan(int b, int hq, int hkv, int s, int d, int
  * process; 0 restores the automatic choice. A forced size that does not fit
  * a shape makes those calls return DS_ERR_UNSUPPORTED. Tuning/testing knob. */
 DS_API void ds_sparse_decode_set_cluster(int n);
+
+/* Process-wide tuning/testing knobs of ds_sparse_decode and the decode
+ * steps (scheduling and prefetch choices; results never depend on them).
+ * A negative value restores the default. DS_ERR_INVALID_ARG for an unknown
+ * name or a value out of range.
+ *   "stagger"       (0..100, default 100) staggered first wave: the second
+ *                   half of the CTAs resident at once holds its label stream
+ *                   back until this percentage of the first half has streamed
+ *                   its label rows (or a poll limit of some tens of
+ *                   microseconds has passed), so one half's selection overlaps
+ *                   the other half's streaming; 0 turns it off. Its counters
+ *                   live in a small array inside the library, shared by
+ *                   concurrent decode launches on a device (which can only
+ *                   delay them up to the poll limit).
+ *   "att_prefetch"  (0..16, default 4) attention: 8-token tiles of selected
+ *                   K/V rows prefetched into L2 ahead of the copy ring.
+ *   "scan_prefetch" (0..8, default 2) label scan through registers (when the
+ *                   shared-memory ring does not fit): rounds of label rows
+ *                   prefetched into L2 ahead. */
+DS_API ds_status ds_sparse_decode_tune(const char* name, int value);
+
+/* Every wait of a kernel on a transaction barrier (a bulk copy landing in
+ * shared memory) polls a bounded number of times. A wait that gives up
+ * records where in a status word inside the library and the kernel leaves
+ * instead of hanging the GPU; the results of that launch are then undefined.
+ * ds_check_device synchronises `stream`, reads the word and clears it:
+ * DS_OK if no wait gave up since the last check, else DS_ERR_TIMEOUT
+ * (ds_last_error names the sites). Not a hot-path call. */
+DS_API ds_status ds_check_device(cudaStream_t stream);
+
+/* Self-test of that mechanism: launches one thread that waits on a
+ * transaction barrier nothing completes, for about `polls` microseconds, so
+ * the wait runs out and is recorded (site bit 0); the next ds_check_device
+ * returns DS_ERR_TIMEOUT. DS_ERR_INVALID_ARG unless 1 <= polls <= 1000000. */
+DS_API ds_status ds_selftest_bounded_wait(int polls, cudaStream_t stream);
 
 /* ------------------------------------------------------------- baseline
  * Dense decode attention over tokens [0, s) of the same cache (no label,

@@ -127,6 +127,52 @@ def test_label_build_and_append_bit_exact(kv, label, d, c):
         assert np.array_equal(got2, r2)
 
 
+@pytest.mark.parametrize("kv,label,d,c", [("bf16", "bf16", 128, 16), ("bf16", "int4", 128, 32),
+                                          ("f32", "f32", 64, 8), ("f32", "int4", 64, 8), ("bf16", "int4", 128, 8),
+                                          ("bf16", "bf16", 64, 64), ("bf16", "int4", 128, 128),
+                                          ("f32", "f32", 128, 32)])
+def test_pipelined_label_build_bit_exact(kv, label, d, c):
+    """Prefill builds large enough for the pipelined (bulk-copy ring) label
+    kernel: every row bit-exact against the oracle, a ragged last block per
+    row, an odd cache capacity, and rows past s left untouched."""
+    wl = synth.custom(b=4, hq=8, hkv=8, d=d, s=5000, c=c, kv_dtype=kv, label_dtype=label,
+                      n_outlier=min(8, c), index=66)
+    di = synth.decode_inputs(wl, s_cap=5003)
+    idx = _idx_random(wl, 9)
+    kd, idxd = to_dev(di.k, kv), torch.from_numpy(idx).cuda()
+    lab, sc, ze = ds.new_label_cache(kd, c, int4=label == "int4")
+    lab.fill_(7 if label == "int4" else 3)
+    if sc is not None:
+        sc.fill_(5); ze.fill_(5)
+    ds.build_label_cache(kd, idxd, wl.s, lab, sc, ze)
+    ds.check_device()
+    got = _host_label(lab, sc, ze, wl)
+    ref = oracle.build_label(di.k, kv, label, idx, wl.s)
+    if label == "int4":
+        for a, b_ in zip(got, ref):
+            assert np.array_equal(a[:, :, : wl.s], b_[:, :, : wl.s])
+        assert np.all(got[0][:, :, wl.s:] == 7) and np.all(got[1][:, :, wl.s:] == 5)
+    else:
+        assert np.array_equal(got[:, :, : wl.s], ref[:, :, : wl.s])
+        assert torch.all(lab[:, :, wl.s:] == 3)
+
+
+def test_bounded_wait_self_test_reports_timeout():
+    """A kernel wait that runs out is recorded and reported, and the context
+    stays usable: a transaction barrier nothing completes, waited on for about
+    50 us; then a normal launch still runs."""
+    ds.check_device()  # clears any earlier record
+    st = ds.lib().ds_selftest_bounded_wait(50, None)
+    assert st == ds.DS_OK
+    with pytest.raises(ds.DSError) as e:
+        ds.check_device()
+    assert e.value.status == ds.DS_ERR_TIMEOUT
+    ds.check_device()  # cleared by the read
+    x = torch.arange(1024, device="cuda", dtype=torch.float32)
+    assert float(x.sum()) == 1023 * 1024 / 2
+    assert ds.lib().ds_selftest_bounded_wait(0, None) == ds.DS_ERR_INVALID_ARG
+
+
 # ----------------------------------------------------------------- decode
 
 @pytest.mark.parametrize("cluster", [0, 1, 2, 4, 8, 16])

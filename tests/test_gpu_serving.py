@@ -442,3 +442,47 @@ def test_decode_step_kv_equals_copy_then_step(kv, label, cluster):
     assert torch.equal(lab1, lab2) and torch.equal(sel1, sel2) and torch.equal(o1, o2)
     if sc1 is not None:
         assert torch.equal(sc1, sc2) and torch.equal(ze1, ze2)
+
+
+@pytest.mark.parametrize("kv,label,cluster,out_dtype", [("bf16", "bf16", 0, "bf16"), ("bf16", "int4", 4, "f32"),
+                                                        ("f32", "f32", 2, "f32")])
+def test_decode_step_kv_from_host_buffers(kv, label, cluster, out_dtype):
+    """A decode step straight from pinned host buffers: the kernel reads the
+    query and the new token's K/V rows over the host link and writes the
+    output there, giving the same bits as the step on device copies."""
+    b, hq, hkv, d, c, s, topk = 2, 8, 4, 128 if kv == "bf16" else 64, 16, 3000, 200
+    if label == "int4":
+        c = 32
+    if kv == "f32":
+        c = 8
+    wl = synth.custom(b=b, hq=hq, hkv=hkv, d=d, s=s, c=c, topk=topk, kv_dtype=kv, label_dtype=label,
+                      n_outlier=min(16, c), outlier_scale=6.0, index=87)
+    di = synth.decode_inputs(wl, s_cap=s + 8)
+    idxd = torch.from_numpy(_idx_random(wl, 15)).cuda()
+    qd, kd, vd = (to_dev(x, kv) for x in (di.q, di.k, di.v))
+    k_new, v_new = kd[:, :, s - 1].clone(), vd[:, :, s - 1].clone()
+    odt = torch.bfloat16 if out_dtype == "bf16" else torch.float32
+    caches = []
+    for _ in range(2):
+        k1, v1 = kd.clone(), vd.clone()
+        k1[:, :, s - 1] = 0
+        v1[:, :, s - 1] = 0
+        lab, sc, ze = _label_alloc(kd, wl)
+        ds.build_label_cache(kd, idxd, s - 1, lab, sc, ze)
+        caches.append((k1, v1, lab, sc, ze))
+    qh, knh, vnh = (t.cpu().pin_memory() for t in (qd, k_new, v_new))
+    oh = torch.full((b, hq, d), float("nan"), dtype=odt).pin_memory()
+    od = torch.empty((b, hq, d), dtype=odt, device="cuda")
+    ds.set_cluster(cluster)
+    try:
+        k1, v1, lab, sc, ze = caches[0]
+        ds.decode_step_kv(qh, knh, vnh, k1, v1, lab, idxd, s, topk, lscale=sc, lzero=ze, out=oh)
+        k2, v2, lab2, sc2, ze2 = caches[1]
+        ds.decode_step_kv(qd, k_new, v_new, k2, v2, lab2, idxd, s, topk, lscale=sc2, lzero=ze2, out=od)
+        torch.cuda.synchronize()
+    finally:
+        ds.set_cluster(0)
+    assert torch.equal(k1, k2) and torch.equal(v1, v2) and torch.equal(lab, lab2)
+    assert torch.equal(oh, od.cpu())
+    with pytest.raises(ValueError):  # pageable host memory is refused
+        ds.decode_step_kv(qd.cpu(), k_new, v_new, k1, v1, lab, idxd, s, topk, lscale=sc, lzero=ze, out=od)

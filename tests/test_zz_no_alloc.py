@@ -1,8 +1,7 @@
 """The allocation-free calibration entry point.
 
-Some callers cannot allocate device memory: code running while a CUDA graph
-is captured, plugins whose host framework owns every allocation, or runtimes
-with a fixed device budget. ds_calibrate_channels_noalloc serves them with a
+Some callers cannot allocate device memory: plugins whose host framework
+owns every allocation, or runtimes with a fixed device budget. ds_calibrate_channels_noalloc serves them with a
 fixed scratch array inside the library instead of a caller workspace. This
 test calls it through the C ABI twice in a row (the shared scratch keeps the
 previous call's contents, so the second call checks that it is cleared) and
@@ -73,6 +72,28 @@ def test_noalloc_matches_workspace_entry_point_twice(index, hq, hkv, d, c, s, n_
         torch.cuda.synchronize()
         assert torch.equal(idx, idx_ref)
         np.testing.assert_allclose(ratio.cpu().numpy(), ratio_ref.cpu().numpy(), rtol=2e-5, atol=1e-7)
+
+
+def test_noalloc_call_takes_no_device_memory():
+    """After a first call (which looks up the scratch array's address), calls
+    change neither torch's allocations nor the device's free memory."""
+    wl, q_win, k = _inputs(83, 8, 4, 128, 16, 512, 2, "bf16")
+    idx, ratio = _noalloc(q_win, k, 16)  # first call in this context
+    torch.cuda.synchronize()
+    alloc0 = torch.cuda.memory_allocated()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        n, hq, w, d = q_win.shape
+        _, hkv, s, _ = k.shape
+        st = ds.lib().ds_calibrate_channels_noalloc(
+            C.c_void_p(q_win.data_ptr()), C.c_void_p(k.data_ptr()), ds.DS_BF16, n, hq, hkv, w, s, d, 16,
+            C.c_void_p(ratio.data_ptr()), C.c_void_p(idx.data_ptr()),
+            C.c_void_p(torch.cuda.current_stream().cuda_stream))
+        assert st == ds.DS_OK, ds.last_error()
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert torch.cuda.memory_allocated() == alloc0
+    assert free1 == free0
 
 
 def test_noalloc_rejects_problems_beyond_the_fixed_scratch():
