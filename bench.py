@@ -725,6 +725,8 @@ def main():
                     help="rows per reference-arm step (0: one per host thread)")
     ap.add_argument("--label", default=None, choices=["f32", "bf16", "int4"],
                     help="override the headline workload's label cache dtype (measurement variants)")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the headline workload's batch (smaller cases for profiling)")
     ap.add_argument("--offload", action="store_true",
                     help="also time the step with the K/V caches in pinned host memory")
     ap.add_argument("--timing", default="rotate", choices=["rotate", "flush"],
@@ -743,6 +745,8 @@ def main():
         if args.label != "int4" and args.label != wl.kv_dtype:
             raise SystemExit("an fp label cache has the key cache's dtype")
         wl = dataclasses.replace(wl, label_dtype=args.label, name=f"{wl.name}, {args.label} label")
+    if args.batch and args.batch != wl.b:
+        wl = dataclasses.replace(wl, b=args.batch, name=wl.name.replace(f"b{wl.b} ", f"b{args.batch} ", 1))
     rank, local_rank, world = dist_env()
 
     if args.impl == "reference":

@@ -18,8 +18,8 @@ namespace {
 thread_local char g_err[256] = "";
 std::atomic<int> g_cluster_override{0};
 // Tuning knobs (ds_sparse_decode_tune)
-std::atomic<int> g_stagger_pct{100};  // share of the first group a held-back CTA waits for (0: off)
-std::atomic<int> g_att_prefetch{4};   // attention: tiles prefetched into L2 ahead of the copy ring
+std::atomic<int> g_stagger_pct{0};  // share of the first group a held-back CTA waits for (0: off)
+std::atomic<int> g_att_prefetch{0};   // attention: tiles prefetched into L2 ahead of the copy ring
 std::atomic<int> g_scan_prefetch{2};  // label scan without the ring: rounds prefetched into L2 ahead
 
 // Small device words of the library: [0], [1] the counters of the decode
@@ -402,10 +402,10 @@ ds_status ds_sparse_decode_tune(const char* name, int value) {
     const std::string n(name);
     if (n == "stagger") {
         if (value > 100) return fail(DS_ERR_INVALID_ARG, "stagger is a percentage (0..100, <0 default)");
-        g_stagger_pct.store(value < 0 ? 100 : value);
+        g_stagger_pct.store(value < 0 ? 0 : value);
     } else if (n == "att_prefetch") {
         if (value > 16) return fail(DS_ERR_INVALID_ARG, "att_prefetch: 0..16 tiles (<0 default)");
-        g_att_prefetch.store(value < 0 ? 4 : value);
+        g_att_prefetch.store(value < 0 ? 0 : value);
     } else if (n == "scan_prefetch") {
         if (value > 8) return fail(DS_ERR_INVALID_ARG, "scan_prefetch: 0..8 rounds (<0 default)");
         g_scan_prefetch.store(value < 0 ? 2 : value);

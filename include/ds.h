@@ -325,16 +325,16 @@ DS_API void ds_sparse_decode_set_cluster(int n);
  * steps (scheduling and prefetch choices; results never depend on them).
  * A negative value restores the default. DS_ERR_INVALID_ARG for an unknown
  * name or a value out of range.
- *   "stagger"       (0..100, default 100) staggered first wave: the second
+ *   "stagger"       (0..100, default 0 = off) staggered first wave: the second
  *                   half of the CTAs resident at once holds its label stream
  *                   back until this percentage of the first half has streamed
  *                   its label rows (or a poll limit of some tens of
  *                   microseconds has passed), so one half's selection overlaps
- *                   the other half's streaming; 0 turns it off. Its counters
+ *                   the other half's streaming. Its counters
  *                   live in a small array inside the library, shared by
  *                   concurrent decode launches on a device (which can only
  *                   delay them up to the poll limit).
- *   "att_prefetch"  (0..16, default 4) attention: 8-token tiles of selected
+ *   "att_prefetch"  (0..16, default 0) attention: 8-token tiles of selected
  *                   K/V rows prefetched into L2 ahead of the copy ring.
  *   "scan_prefetch" (0..8, default 2) label scan through registers (when the
  *                   shared-memory ring does not fit): rounds of label rows

@@ -353,12 +353,23 @@ def _full_config(i, rows_to_check, label_dtype=None):
     out = ds.sparse_decode(q, k, v, lab, idxd, wl.s, wl.topk, lscale=sc, lzero=ze, sel_out=sel,
                            score_out=scores, out_dtype=torch.float32)
     torch.cuda.synchronize()
+    ds.check_device()
     G = wl.g
+    if rows_to_check == "all":
+        rows_to_check = [(b, g) for b in range(wl.b) for g in range(wl.hkv)]
+    # caches up to 1 GiB are copied to the host once, larger ones row by row
+    whole = k.numel() * k.element_size() * 2 <= (1 << 30)
+    if whole:
+        kh, vh, qh = (to_host(t, wl.kv_dtype) for t in (k, v, q))
     for (b, g) in rows_to_check:
-        # host copies of this row only
-        kr = to_host(k[b:b + 1, g:g + 1].contiguous(), wl.kv_dtype)
-        vr = to_host(v[b:b + 1, g:g + 1].contiguous(), wl.kv_dtype)
-        qr = to_host(q[b:b + 1, g * G:(g + 1) * G].contiguous(), wl.kv_dtype)
+        if whole:
+            kr = np.ascontiguousarray(kh[b:b + 1, g:g + 1])
+            vr = np.ascontiguousarray(vh[b:b + 1, g:g + 1])
+            qr = np.ascontiguousarray(qh[b:b + 1, g * G:(g + 1) * G])
+        else:
+            kr = to_host(k[b:b + 1, g:g + 1].contiguous(), wl.kv_dtype)
+            vr = to_host(v[b:b + 1, g:g + 1].contiguous(), wl.kv_dtype)
+            qr = to_host(q[b:b + 1, g * G:(g + 1) * G].contiguous(), wl.kv_dtype)
         ir = np.ascontiguousarray(idx[g:g + 1], np.int32)
         ref_lab = oracle.build_label(kr, wl.kv_dtype, wl.label_dtype, ir, wl.s)
         if wl.label_dtype == "int4":
@@ -382,14 +393,25 @@ def _full_config(i, rows_to_check, label_dtype=None):
     assert torch.isfinite(out).all()
 
 
+# Rows of the 32-channel layer (1024 one-CTA rows): both ends, both sides of
+# the staggered first wave's halves (CTAs 0-147 and 148-295 on 148 SMs), the
+# first rows of the later waves, and the middle.
+_C2_ROWS = [divmod(r, 32) for r in (0, 1, 147, 148, 149, 295, 296, 297, 511, 512, 700, 1022, 1023)]
+
+
 @pytest.mark.parametrize("i,rows", [
     (0, None),
-    (1, [(0, 0), (3, 17), (7, 31)]),
-    (2, [(0, 0), (31, 31)]),
-    (3, [(0, 0), (3, 7)]),
-    (4, [(0, 0), (0, 31)]),
+    (1, "all"),
+    (2, _C2_ROWS),
+    (3, "all"),
+    (4, [(0, 0), (0, 1), (0, 15), (0, 16), (0, 30), (0, 31)]),
 ])
 def test_full_size_configs(i, rows):
+    """Every workload at its full size against the oracle: every row of the
+    Llama-2-7B and GQA layers; on the two multi-GB ones, rows spread over the
+    launch (first and last, both halves of the staggered first wave, later
+    waves, the middle). Scores, selection and output row by row; label bits
+    of each checked row."""
     _full_config(i, rows)
 
 
