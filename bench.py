@@ -44,6 +44,7 @@ METRIC = "sparse-decode attn tokens/s per layer; achieved HBM GB/s (% of B200 pe
 UNIT = "tokens/s/layer"
 NOMINAL_HBM_GBS = 8000.0
 FLUSH_BYTES = 512 << 20
+CHAIN_STEPS = 8  # at least this many consecutive steps per captured graph
 KERNEL_SOURCES = ["channel_token_sparse_b200/csrc/ds_decode_kernel.cuh",
                   "channel_token_sparse_b200/csrc/ds_common.cuh",
                   "channel_token_sparse_b200/csrc/ds_decode_bf16_fp.cu",
@@ -311,6 +312,15 @@ def run_ours(args, wl, rank, local_rank, world):
             fn()
         graphs.append(g)
 
+    # consecutive steps (layer instances in turn) are also captured together,
+    # M of them in one graph, as a decode loop launches its layers: the steps
+    # then run back to back without a graph launch between each two
+    M = R * -(-CHAIN_STEPS // R)
+    chain = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(chain, stream=stream):
+        for j in range(M):
+            step_of(states[j % R])()
+
     def one_step(i, evs=None):
         if timing == "flush":
             flush()  # untimed: evicts L2 (the step's inputs could otherwise stay in the 126 MB L2)
@@ -320,9 +330,24 @@ def run_ours(args, wl, rank, local_rank, world):
         if evs:
             evs[1].record()
 
+    def run_steps(start, count):
+        """Launch exactly `count` steps, instances start % R, (start + 1) % R, ..."""
+        i, end = start, start + count
+        while i < end and i % M:
+            graphs[i % R].replay()
+            i += 1
+        while i + M <= end:
+            chain.replay()
+            i += M
+        while i < end:
+            graphs[i % R].replay()
+            i += 1
+
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
             one_step(i)
+        if timing != "flush":
+            chain.replay()  # warm the chained graph too
     torch.cuda.synchronize()
 
     sampler = ClockSampler(local_rank)
@@ -346,8 +371,7 @@ def run_ours(args, wl, rank, local_rank, world):
             wall0 = time.perf_counter()
             with torch.cuda.stream(stream):
                 t0.record()
-                for i in range(args.steps):
-                    one_step(args.warmup + i)
+                run_steps(args.warmup, args.steps)
                 t1.record()
             torch.cuda.synchronize()
             wall1 = time.perf_counter()
@@ -400,7 +424,7 @@ def run_ours(args, wl, rank, local_rank, world):
     dense_ms, sdpa_ms = dense_baselines(wl, q, k, v, out, flush if timing == "flush" else None, stream)
     offload = offload_timing(wl, q, k, v, idx, lab, sc, ze, out, flush, stream) if args.offload else None
 
-    res = dict(step_ms=step_ms, total_s=total_s, max_s=max_s, timing=timing, rotate=R,
+    res = dict(step_ms=step_ms, total_s=total_s, max_s=max_s, timing=timing, rotate=R, chain=M,
                wall_s=wall1 - wall0, e2e_s=e2e_max, h2d=h2d, d2h=d2h, prefill_ms=prefill_ms,
                clocks=sampler.summary(), dense_ms=dense_ms, sdpa_ms=sdpa_ms, offload=offload,
                plan=ds.plan(wl.b, wl.hq, wl.hkv, wl.s, wl.d, wl.c, wl.topk,
@@ -796,7 +820,8 @@ def l2_note(args, r) -> str:
     if r["timing"] == "rotate":
         return (f"inputs larger than L2: the {args.steps} timed steps run back to back, cycling through "
                 f"{r['rotate']} independent layer instances (own q, K, V, label cache and output) whose "
-                f"working sets together exceed twice the L2; one event pair around the K steps")
+                f"working sets together exceed twice the L2, launched as CUDA graphs of {r['chain']} "
+                f"consecutive steps; one event pair around the K steps")
     return (f"flushed before every timed step: {FLUSH_BYTES >> 20} MiB written by "
             + ("a device-to-device copy" if args.flush == "copy" else "a fill kernel")
             + (f", then {FLUSH_BYTES >> 20} MiB read (flush data written back before the step)"

@@ -17,25 +17,18 @@ namespace {
 
 thread_local char g_err[256] = "";
 std::atomic<int> g_cluster_override{0};
-// Tuning knobs (ds_sparse_decode_tune)
-std::atomic<int> g_stagger_pct{0};  // share of the first group a held-back CTA waits for (0: off)
-std::atomic<int> g_att_prefetch{0};   // attention: tiles prefetched into L2 ahead of the copy ring
+// Tuning knob (ds_sparse_decode_tune)
 std::atomic<int> g_scan_prefetch{2};  // label scan without the ring: rounds prefetched into L2 ahead
+std::atomic<int> g_i4_ring{0};        // 4-bit rows: 1 = the label ring before the kept low key bits
 
-// Small device words of the library: [0], [1] the counters of the decode
-// kernel's staggered first wave (see DecodeParams; the kernel's last CTA
-// resets them, so every launch finds them at zero; concurrent decode launches
-// on one device share them, which can only delay a held-back CTA up to its
-// poll limit, never change a result); [2] the status word in which a kernel
-// records a bounded wait that gave up (bit = where; read and cleared by
-// ds_check_device).
-static __device__ __align__(16) unsigned int g_decode_sched[4];
-constexpr int kStatusWord = 2;
+// The library's status word on each device: a kernel records there a
+// bounded wait that gave up (bit = where); ds_check_device reads and clears it.
+static __device__ __align__(16) unsigned int g_status_word[4];
 
-std::mutex g_sched_mu;
-struct SchedAddr { unsigned long long ctx; unsigned int* ptr; };
-SchedAddr g_sched_addr[16];
-int g_sched_used = 0, g_sched_next = 0;
+std::mutex g_status_mu;
+struct StatusAddr { unsigned long long ctx; unsigned int* ptr; };
+StatusAddr g_status_addr[16];
+int g_status_used = 0, g_status_next = 0;
 
 ds_status fail(ds_status st, const char* fmt, ...) {
     va_list ap;
@@ -121,8 +114,13 @@ bool make_plan(int rows, int G, int s, int d, int c, int topk, bool dense, bool 
         p.lab_ring = 0;
         p.keep_low = 0;
         if (!dense) {
+            // The selection phase keeps the 16-bit keys, optionally the low
+            // 16 key bits, and the label ring in the region the attention
+            // ring uses later; the region may grow beyond the attention ring
+            // for them, as long as the CTAs per SM the plan has stay resident.
             const ds::DecodeSmem L = ds::decode_smem_layout(GT, d, c, p.lay_chunk, p.per, esz, p.att_stages);
-            const int region = L.total - L.region;
+            const int region_att = L.total - L.region;
+            const int cap = (L.total <= kSmemFor2 ? kSmemFor2 : kMaxSmem) - L.region;
             const int keys = ds::align16(p.lay_chunk * 2);
             // 4-bit rows also stream their fp16 scale and zero in 16-byte
             // chunks of 8 tokens, which needs rows of a multiple of 8 tokens
@@ -130,17 +128,24 @@ bool make_plan(int rows, int G, int s, int d, int c, int topk, bool dense, bool 
             const bool i4_ring = int4 && s_cap > 0 && s_cap % 8 == 0 && (pay == 4 || pay == 8 || pay % 16 == 0);
             const int ring = int4 ? (i4_ring ? ds::lab_ring_bytes(pay + 4) : -1)
                                   : ((c * esz) % 16 == 0 ? ds::lab_ring_bytes(c * esz) : -1);
-            // (for 4-bit rows, whose re-scoring costs more, the kept low
-            // bits come before the ring when only one of them fits)
-            if (ring >= 0 && 2 * keys + ring <= region) {
-                p.lab_ring = 1;
-                p.keep_low = 1;
-            } else if (ring >= 0 && keys + ring <= region && !int4) {
-                p.lab_ring = 1;
-            } else if (2 * keys <= region) {
-                p.keep_low = 1;
-            } else if (ring >= 0 && keys + ring <= region) {
-                p.lab_ring = 1;
+            // options in order of preference: {bytes, ring, low}; for 4-bit
+            // rows, whose re-scoring costs more, the kept low bits come before
+            // the ring when only one of them fits
+            struct Opt { int need, ring, low; };
+            const bool ring_first = !int4 || g_i4_ring.load();
+            const Opt opts[] = {
+                {ring >= 0 ? 2 * keys + ring : -1, 1, 1},
+                {ring >= 0 && ring_first ? keys + ring : -1, 1, 0},
+                {2 * keys, 0, 1},
+                {ring >= 0 ? keys + ring : -1, 1, 0},
+            };
+            for (const Opt& o : opts) {
+                if (o.need < 0 || o.need > cap) continue;
+                p.lab_ring = o.ring;
+                p.keep_low = o.low;
+                if (o.need > region_att)
+                    p.smem = ds::decode_smem_layout(GT, d, c, p.lay_chunk, p.per, esz, p.att_stages, o.need).total;
+                break;
             }
         }
         if (forced) {
@@ -252,44 +257,25 @@ __global__ void ds_selftest_wait_kernel(unsigned int* err, unsigned long long li
     if (threadIdx.x == 0) ds::mbar_wait_bounded(&bar, 0, err, 0, limit_ns);
 }
 
-// Device address of g_decode_sched in the current context, cached per
+// Device address of g_status_word in the current context, cached per
 // context (host code only has the array's name as a host-side stand-in).
-cudaError_t sched_counters(unsigned int** out) {
+cudaError_t status_word(unsigned int** out) {
     unsigned long long ctx = 0;
     const bool keyed = ds::current_context_id(&ctx);
-    std::lock_guard<std::mutex> lk(g_sched_mu);
+    std::lock_guard<std::mutex> lk(g_status_mu);
     if (keyed)
-        for (int i = 0; i < g_sched_used; ++i)
-            if (g_sched_addr[i].ctx == ctx) { *out = g_sched_addr[i].ptr; return cudaSuccess; }
+        for (int i = 0; i < g_status_used; ++i)
+            if (g_status_addr[i].ctx == ctx) { *out = g_status_addr[i].ptr; return cudaSuccess; }
     void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_sched);
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_status_word);
     if (e != cudaSuccess) return e;
     if (keyed || ds::current_context_id(&ctx)) {
-        g_sched_addr[g_sched_next] = SchedAddr{ctx, static_cast<unsigned int*>(p)};
-        g_sched_next = (g_sched_next + 1) % 16;
-        if (g_sched_used < 16) ++g_sched_used;
+        g_status_addr[g_status_next] = StatusAddr{ctx, static_cast<unsigned int*>(p)};
+        g_status_next = (g_status_next + 1) % 16;
+        if (g_status_used < 16) ++g_status_used;
     }
     *out = static_cast<unsigned int*>(p);
     return cudaSuccess;
-}
-
-// Staggered first wave: of the CTAs resident at once, the first half (whole
-// clusters) streams its label rows at once, the second half waits for it
-// (see DecodeParams). Rows that only fill part of a wave, or fewer than two
-// clusters, are not staggered.
-ds_status plan_stagger(ds::DecodeParams& p, int rows, int N, int slots) {
-    p.sched = nullptr;
-    const int pct = g_stagger_pct.load();
-    const int grid = rows * N;
-    const int wave = (grid < slots ? grid : slots) / N * N;
-    if (pct <= 0 || wave < 2 * N) return DS_OK;
-    cudaError_t e = sched_counters(&p.sched);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
-    p.stagger_a = wave / 2 / N * N;
-    p.stagger_end = wave;
-    p.stagger_target = (p.stagger_a * pct + 99) / 100;
-    p.stagger_polls = 400;  // ~40-80 us of __nanosleep(100) at most
-    return DS_OK;
 }
 
 ds_status check_common(int b, int hq, int hkv, int s, int s_cap, int d, ds_dtype kvdt) {
@@ -361,9 +347,9 @@ ds_status run_label(const void* k, ds_dtype kdt, const int32_t* idx, int b, int 
                     label, lscale, lzero};
     unsigned int* words = nullptr;
     if (!pg && t_end - t_begin > 1) {
-        cudaError_t e = sched_counters(&words);
+        cudaError_t e = status_word(&words);
         if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
-        a.err = words + kStatusWord;
+        a.err = words;
         a.sms = sm_count();
     }
     if (pg) {
@@ -400,15 +386,12 @@ void ds_sparse_decode_set_cluster(int n) { g_cluster_override.store(n); }
 ds_status ds_sparse_decode_tune(const char* name, int value) {
     if (!name) return fail(DS_ERR_INVALID_ARG, "name is NULL");
     const std::string n(name);
-    if (n == "stagger") {
-        if (value > 100) return fail(DS_ERR_INVALID_ARG, "stagger is a percentage (0..100, <0 default)");
-        g_stagger_pct.store(value < 0 ? 0 : value);
-    } else if (n == "att_prefetch") {
-        if (value > 16) return fail(DS_ERR_INVALID_ARG, "att_prefetch: 0..16 tiles (<0 default)");
-        g_att_prefetch.store(value < 0 ? 0 : value);
-    } else if (n == "scan_prefetch") {
+    if (n == "scan_prefetch") {
         if (value > 8) return fail(DS_ERR_INVALID_ARG, "scan_prefetch: 0..8 rounds (<0 default)");
         g_scan_prefetch.store(value < 0 ? 2 : value);
+    } else if (n == "i4_ring") {
+        if (value > 1) return fail(DS_ERR_INVALID_ARG, "i4_ring: 0 or 1 (<0 default)");
+        g_i4_ring.store(value < 0 ? 0 : value);
     } else {
         return fail(DS_ERR_INVALID_ARG, "unknown tuning knob '%s'", name);
     }
@@ -418,9 +401,9 @@ ds_status ds_sparse_decode_tune(const char* name, int value) {
 ds_status ds_selftest_bounded_wait(int polls, cudaStream_t stream) {
     if (polls < 1 || polls > 1000000) return fail(DS_ERR_INVALID_ARG, "polls must be in [1, 1000000]");
     unsigned int* words = nullptr;
-    cudaError_t e = sched_counters(&words);
+    cudaError_t e = status_word(&words);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
-    ds_selftest_wait_kernel<<<1, 32, 0, stream>>>(words + kStatusWord, (unsigned long long)polls * 1000ull);
+    ds_selftest_wait_kernel<<<1, 32, 0, stream>>>(words, (unsigned long long)polls * 1000ull);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
     return DS_OK;
@@ -428,15 +411,15 @@ ds_status ds_selftest_bounded_wait(int polls, cudaStream_t stream) {
 
 ds_status ds_check_device(cudaStream_t stream) {
     unsigned int* words = nullptr;
-    cudaError_t e = sched_counters(&words);
+    cudaError_t e = status_word(&words);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
     unsigned int w = 0;
-    e = cudaMemcpyAsync(&w, words + kStatusWord, sizeof w, cudaMemcpyDeviceToHost, stream);
+    e = cudaMemcpyAsync(&w, words, sizeof w, cudaMemcpyDeviceToHost, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return cuda_fail(e, "reading the device status");
     if (!w) return DS_OK;
     const unsigned int zero = 0;
-    e = cudaMemcpyAsync(words + kStatusWord, &zero, sizeof zero, cudaMemcpyHostToDevice, stream);
+    e = cudaMemcpyAsync(words, &zero, sizeof zero, cudaMemcpyHostToDevice, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the device status");
     return fail(DS_ERR_TIMEOUT, "a kernel gave up a bounded wait (sites 0x%x: bit 0 self-test, "
@@ -629,8 +612,6 @@ ds_status sparse_decode_impl(const void* q, const void* k, const void* v, ds_dty
     p.qscale = scale * 1.4426950408889634f;
     p.out_bf16 = out_dt == DS_BF16;
     p.dense = 0;
-    if ((r = plan_stagger(p, rows, pl.N, kCtasPerSm * sm_count())) != DS_OK) return r;
-    p.att_prefetch = g_att_prefetch.load();
     p.scan_prefetch = g_scan_prefetch.load();
     return launch_decode(kern, p, rows, pl, stream);
 }

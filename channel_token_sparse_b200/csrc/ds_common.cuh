@@ -112,6 +112,21 @@ __device__ __forceinline__ void lds_row(uint32_t (&w)[N / 4], const uint8_t* p) 
     }
 }
 
+// The 4-bit code of value x with zero z and scale sc > 0:
+// clamp(rint((x - z) / sc), 0, 15), the quotient an IEEE single-precision
+// division rounded to nearest even. The quotient is first formed as
+// (x - z) * (1 / sc), within 3 * 2^-24 relative of the exact one; rint can only
+// differ between the two when a half-integer lies within that distance, so
+// only then (|frac - 1/2| <= 1e-5, codes < 16 keep |q| <= 16) is the division
+// done exactly. The result is always that of the exact division.
+__device__ __forceinline__ uint32_t int4_code(float x, float z, float sc, float rcp_sc) {
+    const float a = __fsub_rn(x, z);
+    float q = __fmul_rn(a, rcp_sc);
+    if (fabsf(q - floorf(q) - 0.5f) <= 1e-5f) q = __fdiv_rn(a, sc);
+    q = fminf(fmaxf(rintf(q), 0.f), 15.f);
+    return (uint32_t)q;
+}
+
 // 4-bit label row of one token (the heavy channels idx[0..c) of key row x):
 // in fp32, mn/mx over the c values, scale = fp16_rn((mx - mn) / 15),
 // zero = fp16_rn(mn), code_j = scale > 0 ? clamp(rint((x_j - zero) / scale),
@@ -285,15 +300,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                  ::"r"(smem_u32(smem_dst)), "l"(gsrc), "r"(bytes), "r"(smem_u32(bar)) : "memory");
-}
-
-// Named barrier over `nthreads` threads (a multiple of 32) of the CTA;
-// id 0 is __syncthreads'.
-__device__ __forceinline__ void named_sync(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-__device__ __forceinline__ void named_arrive(int id, int nthreads) {
-    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // Two floats -> packed bf16x2 (first in the low half), round to nearest even.

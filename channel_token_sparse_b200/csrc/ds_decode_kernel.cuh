@@ -75,19 +75,8 @@ struct DecodeParams {
     // the kernel writes them into the K/V caches at position s-1 itself
     const void* k_new;
     const void* v_new;
-    // Staggered start of the first wave (a scheduling hint; results never
-    // depend on it). CTAs [0, stagger_a) stream their label rows at once and
-    // count themselves in sched[0] when done; CTAs [stagger_a, stagger_end)
-    // hold back their label stream until sched[0] >= stagger_target or
-    // stagger_polls polls have passed, so that their scan overlaps the
-    // selection of the first group instead of coinciding with it. sched[1]
-    // counts finished CTAs; the last one resets both for the next launch.
-    // sched == null disables it.
-    unsigned int* sched;
-    int stagger_a, stagger_end, stagger_target, stagger_polls;
-    // L2 prefetch distances: attention tiles ahead of the copy ring; label
-    // rounds ahead of the register-path scan (0: none)
-    int att_prefetch, scan_prefetch;
+    // label rounds pulled into L2 ahead of the register-path scan (0: none)
+    int scan_prefetch;
 };
 
 // Row (in units of d elements) of token t of (b, g) in the K/V caches, dense
@@ -130,8 +119,10 @@ __host__ __device__ constexpr int att_ring_bytes(int row_bytes, int elem_bytes, 
 constexpr int kBucketCap = 1024;
 constexpr int kMaxCluster = 16;  // CTAs per row at most (portable 8, non-portable 16)
 
+// region_min: room the selection phase wants for the label ring and the
+// low key bits beyond the keys and the attention ring (host plans only).
 __host__ __device__ inline DecodeSmem decode_smem_layout(int GT, int D, int C, int chunk, int per,
-                                                         int elem_bytes, int att_stages) {
+                                                         int elem_bytes, int att_stages, int region_min = 0) {
     DecodeSmem L;
     int o = 0;
     L.qs = o;     o += align16(GT * D * 4);
@@ -153,7 +144,9 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int GT, int D, int C, i
     L.region = o;
     const int keys = chunk * 2;
     const int ring = kNW * att_ring_bytes(D * elem_bytes, elem_bytes, att_stages);
-    o += align16(keys > ring ? keys : ring);
+    int region = keys > ring ? keys : ring;
+    if (region_min > region) region = region_min;
+    o += align16(region);
     L.total = o;
     return L;
 }
@@ -392,14 +385,6 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
             }
         }
     };
-    const bool stagger_b = p.sched && (int)blockIdx.x >= p.stagger_a && (int)blockIdx.x < p.stagger_end;
-    if (stagger_b) {
-        if (tid == 0) {
-            const volatile unsigned int* cnt = p.sched;
-            for (int i = 0; i < p.stagger_polls && *cnt < (unsigned int)p.stagger_target; ++i) __nanosleep(100);
-        }
-        __syncthreads();
-    }
     if (use_ring) {
 #pragma unroll 1
         for (int j = 0; j < kLabStages - 1; ++j) { issue(j); cp_async_commit(); }
@@ -590,10 +575,6 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     constexpr int RB = D * E::kBytes;              // bytes of one K or V row
     int T16 = 0, Tlo = 0, r_tie = 0;
     bool refine = false;
-    if (p.sched && (int)blockIdx.x < p.stagger_a) {
-        __syncthreads();                                             // this CTA's label scan is done
-        if (tid == 0) atomicAdd(p.sched, 1u);
-    }
     if (!select_all) {
         row_sync(cluster, N);                                        // histograms A complete
         cluster_select_bin(cluster, histA, N, (uint32_t)k_eff, ctl, scan, nullptr);
@@ -987,19 +968,6 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
                 if (bi < nb) issue_stage(bi);
                 cp_async_commit();
             }
-            // tiles further ahead are pulled into L2: lane l takes 128-byte
-            // line l & 1 of the K (l < 16) or V row of token (l >> 1) & 7
-            const int apf = p.att_prefetch;
-            auto prefetch_tile = [&](int bi) {
-                const int u = (lane >> 1) & 7;
-                const int bt0 = (wid + bi * kNW) * TB8;
-                if (bi < nb && bt0 + u < n_att) {
-                    const TKV* base = lane < 16 ? kb : vb;
-                    prefetch_line_l2(reinterpret_cast<const uint8_t*>(base + att_row(bt0 + u) * D) + ((lane & 1) << 7));
-                }
-            };
-            if (RB == 256)
-                for (int bi = stages - 1; bi < stages - 1 + apf; ++bi) prefetch_tile(bi);
             // Q fragments (A operand, rows = heads): bf16 pairs, exact (q is bf16),
             // kept in shared memory ([D/16 steps][32 lanes][2 words]) to spare registers
             const int hr = lane >> 2, kc = (lane & 3) * 2;
@@ -1011,7 +979,6 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
             // [phase] 21
     #pragma unroll 1
             for (int bi = 0; bi < nb; ++bi) {
-                if (RB == 256 && apf > 0) prefetch_tile(bi + stages - 1 + apf);
                 if (bi + stages - 1 < nb) issue_stage(bi + stages - 1);
                 cp_async_commit();
                 if (stages == 3) cp_async_wait<2>();
@@ -1259,17 +1226,6 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
                 Lsum = fmaf(f, cl[r * GT + h], Lsum);
             }
             write_out(h, d, O / Lsum);
-        }
-    }
-    if (p.sched) {
-        // the last CTA to finish resets the stagger counters for the next launch
-        __syncthreads();
-        if (tid == 0) {
-            __threadfence();
-            if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
-                atomicExch(p.sched, 0u);
-                atomicExch(p.sched + 1, 0u);
-            }
         }
     }
     // [phase] 9

@@ -84,7 +84,9 @@ constexpr int kPackLanes = 4;
 
 __host__ __device__ constexpr int bulk_smem_bytes() { return kBulkStages * kBulkStage + kBulkStages * 8; }
 
-template <typename TKV, int LK, int D>
+// CI: the channel count, fixed at compile time for 4-bit rows (each lane's
+// CI / kPackLanes channel indices then stay in registers); 0 for fp rows.
+template <typename TKV, int LK, int D, int CI>
 __global__ void __launch_bounds__(kBulkNT, 2) ds_label_bulk_kernel(const TKV* __restrict__ k,
                                                                   const int32_t* __restrict__ idx, int hkv,
                                                                   int t_begin, int t_end, int s_cap, int c,
@@ -118,9 +120,10 @@ __global__ void __launch_bounds__(kBulkNT, 2) ds_label_bulk_kernel(const TKV* __
             const long long it = blockIdx.x + (long long)i * gridDim.x;
             if (it < items) issue(it, i);
         }
+    constexpr int kPer = CI / kPackLanes > 0 ? CI / kPackLanes : 1;  // 4-bit channels per lane
     int g_cur = -1;
-    int my_idx[128 / kPackLanes > 1 ? 128 / kPackLanes : 1];  // 4-bit: this thread's channels
-    int fp_idx = 0;                                            // fp: this thread's channel (tid % c)
+    int my_idx[kPer];  // 4-bit: this thread's channels
+    int fp_idx = 0;    // fp: this thread's channel (tid % c)
     int j = 0;
     for (long long it = blockIdx.x; it < items; it += gridDim.x, ++j) {
         const int slot = j % kBulkStages;
@@ -134,8 +137,10 @@ __global__ void __launch_bounds__(kBulkNT, 2) ds_label_bulk_kernel(const TKV* __
             if constexpr (LK == 0) {
                 fp_idx = min(max(__ldg(idx + (size_t)g * c + tid % c), 0), D - 1);
             } else {
-                const int per = c / kPackLanes, q = tid % kPackLanes;
-                for (int e = 0; e < per; ++e) my_idx[e] = min(max(__ldg(idx + (size_t)g * c + q * per + e), 0), D - 1);
+                const int q = tid % kPackLanes;
+#pragma unroll
+                for (int e = 0; e < kPer; ++e)
+                    my_idx[e] = min(max(__ldg(idx + (size_t)g * CI + q * kPer + e), 0), D - 1);
             }
         }
         const bool ok = mbar_wait_bounded(&full[slot], (uint32_t)((j / kBulkStages) & 1), err, 1);
@@ -149,12 +154,13 @@ __global__ void __launch_bounds__(kBulkNT, 2) ds_label_bulk_kernel(const TKV* __
                 // kPackLanes threads per token, c / kPackLanes channels each:
                 // the arithmetic of pack_int4_row, with mn / mx combined over
                 // the lanes (fminf / fmaxf do not depend on the order)
-                const int per = c / kPackLanes, q = tid % kPackLanes;
+                const int q = tid % kPackLanes;
                 for (int t = tid / kPackLanes; t < ((nt + 7) & ~7); t += kBulkNT / kPackLanes) {
                     const bool live = t < nt;
                     const TKV* x = rows_s + (size_t)(live ? t : 0) * D;
                     float mn = E::to_f32(x[my_idx[0]]), mx = mn;
-                    for (int e = 1; e < per; ++e) {
+#pragma unroll
+                    for (int e = 1; e < kPer; ++e) {
                         const float v = E::to_f32(x[my_idx[e]]);
                         mn = fminf(mn, v);
                         mx = fmaxf(mx, v);
@@ -168,20 +174,15 @@ __global__ void __launch_bounds__(kBulkNT, 2) ds_label_bulk_kernel(const TKV* __
                     const uint16_t sh = __half_as_ushort(__float2half_rn(step));
                     const uint16_t zh = __half_as_ushort(__float2half_rn(mn));
                     const float sc = fp16_bits_to_f32(sh), z = fp16_bits_to_f32(zh);
+                    const float rsc = sc > 0.f ? __frcp_rn(sc) : 0.f;
                     if (live) {
-                        uint8_t* dst = label + (tok0 + t) * (size_t)(c / 2) + q * per / 2;
-                        for (int e = 0; e < per; e += 2) {
+                        uint8_t* dst = label + (tok0 + t) * (size_t)(CI / 2) + q * kPer / 2;
+#pragma unroll
+                        for (int e = 0; e < kPer; e += 2) {
                             uint32_t nib[2];
 #pragma unroll
-                            for (int h = 0; h < 2; ++h) {
-                                uint32_t code = 0;
-                                if (sc > 0.f) {
-                                    float qv = rintf(__fdiv_rn(__fsub_rn(E::to_f32(x[my_idx[e + h]]), z), sc));
-                                    qv = fminf(fmaxf(qv, 0.f), 15.f);
-                                    code = (uint32_t)qv;
-                                }
-                                nib[h] = code;
-                            }
+                            for (int h = 0; h < 2; ++h)
+                                nib[h] = sc > 0.f ? int4_code(E::to_f32(x[my_idx[e + h]]), z, sc, rsc) : 0u;
                             dst[e / 2] = (uint8_t)(nib[0] | (nib[1] << 4));
                         }
                         if (q == 0) {
@@ -201,25 +202,36 @@ __global__ void __launch_bounds__(kBulkNT, 2) ds_label_bulk_kernel(const TKV* __
     }
 }
 
+template <typename TKV, int LK, int D, int CI>
+static cudaError_t launch_label_bulk(const LabelArgs& a, long long items, cudaStream_t st) {
+    static bool attr = false;  // set once per process (the attribute is per function)
+    if (!attr) {
+        const cudaError_t e = cudaFuncSetAttribute(ds_label_bulk_kernel<TKV, LK, D, CI>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, bulk_smem_bytes());
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    const long long grid = items < 2LL * a.sms ? items : 2LL * a.sms;
+    ds_label_bulk_kernel<TKV, LK, D, CI><<<(unsigned)grid, kBulkNT, bulk_smem_bytes(), st>>>(
+        reinterpret_cast<const TKV*>(a.k), a.idx, a.hkv, a.t_begin, a.t_end, a.s_cap, a.c, a.b * a.hkv,
+        reinterpret_cast<uint8_t*>(a.label), a.lscale, a.lzero, a.err);
+    return cudaGetLastError();
+}
+
 template <typename TKV, int LK, int D>
 static cudaError_t launch_label_t(const LabelArgs& a, cudaStream_t st) {
     const int n = a.t_end - a.t_begin;
     constexpr int kTok = kBulkStage / (D * Elem<TKV>::kBytes);
     const long long items = (long long)a.b * a.hkv * ((n + kTok - 1) / kTok);
     if (!a.block_table && a.err && items >= 2 * (long long)a.sms && (LK == 0 || a.c >= 2 * kPackLanes)) {
-        static bool attr = false;  // set once per process (the attribute is per function)
-        if (!attr) {
-            const cudaError_t e = cudaFuncSetAttribute(ds_label_bulk_kernel<TKV, LK, D>,
-                                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                       bulk_smem_bytes());
-            if (e != cudaSuccess) return e;
-            attr = true;
+        if constexpr (LK == 0) return launch_label_bulk<TKV, 0, D, 0>(a, items, st);
+        switch (a.c) {
+        case 8: return launch_label_bulk<TKV, LK, D, 8>(a, items, st);
+        case 16: return launch_label_bulk<TKV, LK, D, 16>(a, items, st);
+        case 32: return launch_label_bulk<TKV, LK, D, 32>(a, items, st);
+        case 64: if constexpr (D >= 64) return launch_label_bulk<TKV, LK, D, 64>(a, items, st); break;
+        case 128: if constexpr (D >= 128) return launch_label_bulk<TKV, LK, D, 128>(a, items, st); break;
         }
-        const long long grid = items < 2LL * a.sms ? items : 2LL * a.sms;
-        ds_label_bulk_kernel<TKV, LK, D><<<(unsigned)grid, kBulkNT, bulk_smem_bytes(), st>>>(
-            reinterpret_cast<const TKV*>(a.k), a.idx, a.hkv, a.t_begin, a.t_end, a.s_cap, a.c, a.b * a.hkv,
-            reinterpret_cast<uint8_t*>(a.label), a.lscale, a.lzero, a.err);
-        return cudaGetLastError();
     }
     dim3 grid((n + kTokens - 1) / kTokens, a.b * a.hkv);
     ds_label_kernel<TKV, LK, D><<<grid, kLabNT, 0, st>>>(

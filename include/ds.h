@@ -321,24 +321,16 @@ DS_API ds_status ds_sparse_decode_plan(int b, int hq, int hkv, int s, int d, int
  * a shape makes those calls return DS_ERR_UNSUPPORTED. Tuning/testing knob. */
 DS_API void ds_sparse_decode_set_cluster(int n);
 
-/* Process-wide tuning/testing knobs of ds_sparse_decode and the decode
- * steps (scheduling and prefetch choices; results never depend on them).
- * A negative value restores the default. DS_ERR_INVALID_ARG for an unknown
- * name or a value out of range.
- *   "stagger"       (0..100, default 0 = off) staggered first wave: the second
- *                   half of the CTAs resident at once holds its label stream
- *                   back until this percentage of the first half has streamed
- *                   its label rows (or a poll limit of some tens of
- *                   microseconds has passed), so one half's selection overlaps
- *                   the other half's streaming. Its counters
- *                   live in a small array inside the library, shared by
- *                   concurrent decode launches on a device (which can only
- *                   delay them up to the poll limit).
- *   "att_prefetch"  (0..16, default 0) attention: 8-token tiles of selected
- *                   K/V rows prefetched into L2 ahead of the copy ring.
+/* Process-wide tuning/testing knobs of ds_sparse_decode and the decode steps
+ * (prefetch and staging choices; results never depend on them). A negative value restores
+ * the default. DS_ERR_INVALID_ARG for an unknown name or a value out of
+ * range.
  *   "scan_prefetch" (0..8, default 2) label scan through registers (when the
  *                   shared-memory ring does not fit): rounds of label rows
- *                   prefetched into L2 ahead. */
+ *                   prefetched into L2 ahead.
+ *   "i4_ring"       (0 or 1, default 0) 4-bit label rows: when the label ring
+ *                   and the kept low key bits do not both fit, 1 takes the
+ *                   ring (bucket tokens are then re-scored), 0 the low bits. */
 DS_API ds_status ds_sparse_decode_tune(const char* name, int value);
 
 /* Every wait of a kernel on a transaction barrier (a bulk copy landing in
