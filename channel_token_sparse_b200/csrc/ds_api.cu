@@ -19,7 +19,7 @@ thread_local char g_err[256] = "";
 std::atomic<int> g_cluster_override{0};
 // Tuning knob (ds_sparse_decode_tune)
 std::atomic<int> g_scan_prefetch{2};  // label scan without the ring: rounds prefetched into L2 ahead
-std::atomic<int> g_i4_ring{0};        // 4-bit rows: 1 = the label ring before the kept low key bits
+std::atomic<int> g_i4_ring{1};        // 4-bit rows: 1 = the label ring before the kept low key bits
 
 // The library's status word on each device: a kernel records there a
 // bounded wait that gave up (bit = where); ds_check_device reads and clears it.
@@ -391,7 +391,7 @@ ds_status ds_sparse_decode_tune(const char* name, int value) {
         g_scan_prefetch.store(value < 0 ? 2 : value);
     } else if (n == "i4_ring") {
         if (value > 1) return fail(DS_ERR_INVALID_ARG, "i4_ring: 0 or 1 (<0 default)");
-        g_i4_ring.store(value < 0 ? 0 : value);
+        g_i4_ring.store(value < 0 ? 1 : value);
     } else {
         return fail(DS_ERR_INVALID_ARG, "unknown tuning knob '%s'", name);
     }

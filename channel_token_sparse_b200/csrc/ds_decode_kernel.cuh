@@ -91,7 +91,7 @@ __device__ __forceinline__ size_t kv_row_of(const DecodeParams& p, int b, int g,
 
 // Shared-memory carve-up (bytes), identical on host and device.
 struct DecodeSmem {
-    int qs, qa, qL, idx, histA, histB, ctl, scan, cm, cl, co, bits, mcache, blist, app, sel, region, total;
+    int qs, qa, qL, ql4, idx, histA, histB, ctl, scan, cm, cl, co, bits, mcache, blist, app, sel, region, total;
 };
 
 __host__ __device__ inline int align16(int x) { return (x + 15) & ~15; }
@@ -128,6 +128,7 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int GT, int D, int C, i
     L.qs = o;     o += align16(GT * D * 4);
     L.qa = o;     o += elem_bytes == 2 ? (D / 16) * 32 * 8 : 0;  // packed bf16 Q fragments
     L.qL = o;     o += align16(C * 4);
+    L.ql4 = o;    o += align16(C * 3);                      // 4-bit scoring: qL as byte limbs
     L.idx = o;    o += align16(C * 4);
     L.histA = o;  o += 256 * 4;
     L.histB = o;  o += 256 * 4;
@@ -165,33 +166,67 @@ struct LabelGeom {
     static constexpr int kU = (128 / kBytes) < 1 ? 1 : ((128 / kBytes) > 8 ? 8 : (128 / kBytes));
 };
 
+// 4-bit rows: the dot product sum_j qL[j] n_j in integer arithmetic. qL is
+// held in fixed point, Q_j = rint(qL[j] * 2^E) with E chosen per row so that
+// |Q_j| <= 2^21 (22 significant bits, as fine as the fp32 sum needs), split
+// into bytes Q = q2 * 2^16 + q1 * 2^8 + q0 (q0, q1 unsigned, q2 signed). One
+// 32-bit label word holds 8 channels: its low nibbles (channels 2j) and high
+// nibbles (2j + 1) are two vectors of 4 bytes, so each limb costs two dp4a
+// per word and every product is exact; the three limb sums meet in fp32.
+// lim[(2k + h) * C/8 + i] holds limb k of channels 8i + 2b + h in byte b.
+template <int C>
+__device__ __forceinline__ float i4_dot(const uint32_t (&w)[C / 8], const uint32_t* lim, float s_e) {
+    uint32_t s0 = 0u, s1 = 0u;
+    int s2 = 0;
+#pragma unroll
+    for (int i = 0; i < C / 8; ++i) {
+        const uint32_t lo = w[i] & 0x0F0F0F0Fu, hi = (w[i] >> 4) & 0x0F0F0F0Fu;
+        s0 = __dp4a(lim[0 * (C / 8) + i], lo, s0);
+        s0 = __dp4a(lim[1 * (C / 8) + i], hi, s0);
+        s1 = __dp4a(lim[2 * (C / 8) + i], lo, s1);
+        s1 = __dp4a(lim[3 * (C / 8) + i], hi, s1);
+        s2 = __dp4a((int)lim[4 * (C / 8) + i], (int)lo, s2);
+        s2 = __dp4a((int)lim[5 * (C / 8) + i], (int)hi, s2);
+    }
+    const float f = __fmaf_rn((float)s2, 65536.f, __fmaf_rn((float)s1, 256.f, (float)s0));
+    return __fmul_rn(f, s_e);
+}
+
+// Byte limbs of qL for i4_dot (word `wi` of the 6 * C/8), and the scale 2^-E.
+__device__ __forceinline__ float i4_scale_exp(float qmax, float* two_e) {
+    int e = qmax > 0.f ? (int)((__float_as_uint(qmax) >> 23) & 255u) - 127 : 0;
+    int E = 21 - e;
+    E = E < -126 ? -126 : (E > 126 ? 126 : E);
+    *two_e = __uint_as_float((uint32_t)(127 + E) << 23);
+    return __uint_as_float((uint32_t)(127 - E) << 23);
+}
+template <int C>
+__device__ __forceinline__ uint32_t i4_limb_word(const float* qL, float two_e, int wi) {
+    const int k = wi / (2 * (C / 8)), h = (wi / (C / 8)) & 1, i = wi % (C / 8);
+    uint32_t word = 0u;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        const int q = __float2int_rn(__fmul_rn(qL[8 * i + 2 * b + h], two_e));
+        word |= ((uint32_t)(q >> (8 * k)) & 255u) << (8 * b);
+    }
+    return word;
+}
+
 // fp32 score of one token from its label row (step 2). The arithmetic is a
 // fixed chain of fused multiply-adds in channel order, so scoring the same
 // row twice gives bit-identical results.
+// 4-bit rows use i4_dot with the limbs `lim` and scale `s_e` (the fp qL
+// arguments are unused); fp rows use qreg (C <= 32) or qsm.
 template <typename TKV, int LK, int C>
 __device__ __forceinline__ float label_score(const uint32_t (&w)[LabelGeom<TKV, LK, C>::kWords],
                                              const float* qreg, const float* qsm, float sc, float z,
-                                             float qsum) {
+                                             float qsum, const uint32_t* lim, float s_e) {
     constexpr bool kReg = C <= 32;
     auto ql = [&](int j) -> float { return kReg ? qreg[j] : qsm[j]; };
     float acc = 0.f;
     if constexpr (LK == kLabelInt4) {
-        // Nibble e of a word holds channel e. Shifted to bits 19..22 (the
-        // top of the mantissa) and or-ed into 1.0f it gives 1 + n/16 exactly,
-        // so a nibble costs a shift, a mask and an FMA (no conversion):
-        //   sum_j qL[j] n_j = 16 (sum_j qL[j] (1 + n_j/16) - sum_j qL[j])
-#pragma unroll
-        for (int i = 0; i < C / 8; ++i) {
-            const uint32_t x = w[i];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const uint32_t t = 4 * e <= 19 ? (x << (19 - 4 * e)) : (x >> (4 * e - 19));
-                acc = __fmaf_rn(ql(8 * i + e), __uint_as_float((t & 0x00780000u) | 0x3F800000u), acc);
-            }
-        }
-        const float dot = __fmul_rn(16.f, __fsub_rn(acc, qsum));
         // sum_j qL[j] * (sc * n_j + z) = sc * sum_j qL[j] n_j + z * sum_j qL[j]
-        return __fmaf_rn(sc, dot, __fmul_rn(z, qsum));
+        return __fmaf_rn(sc, i4_dot<C>(w, lim, s_e), __fmul_rn(z, qsum));
     } else if constexpr (Elem<TKV>::kBytes == 2) {
 #pragma unroll
         for (int i = 0; i < C / 2; ++i) {
@@ -451,8 +486,11 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     }
     __syncthreads();
 
-    float qreg[C <= 32 ? C : 1];
-    float qsum = 0.f;
+    constexpr bool kI4Score = LK == kLabelInt4;
+    float qreg[(C <= 32 && !kI4Score) ? C : 1];
+    uint32_t qlim[(C <= 32 && kI4Score) ? 6 * C / 8 : 1];   // 4-bit: limbs in registers
+    const uint32_t* lim = (C <= 32) ? qlim : reinterpret_cast<const uint32_t*>(smem + L.ql4);
+    float qsum = 0.f, s_e = 0.f;
 
     // The label row of the appended token (local index app_i, -1 if none) is
     // read from shared memory: this kernel writes it to the label cache and
@@ -477,23 +515,37 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         uint32_t w[LG::kWords];
         float sc = 0.f, z = 0.f;
         load_label(i, w, sc, z);
-        return label_score<TKV, LK, C>(w, qreg, qLs, sc, z, qsum);
+        return label_score<TKV, LK, C>(w, qreg, qLs, sc, z, qsum, lim, s_e);
     };
 
     if (need_scores) {
-        if constexpr (C <= 32) {
+        if constexpr (C <= 32 && !kI4Score) {
 #pragma unroll
             for (int j = 0; j < C; ++j) qreg[j] = qLs[j];
         }
         for (int j = 0; j < C; ++j) qsum += qLs[j];
+        if constexpr (kI4Score) {
+            float qmax = 0.f;
+            for (int j = 0; j < C; ++j) qmax = fmaxf(qmax, fabsf(qLs[j]));
+            float two_e;
+            s_e = i4_scale_exp(qmax, &two_e);
+            if constexpr (C <= 32) {
+#pragma unroll
+                for (int wi = 0; wi < 6 * C / 8; ++wi) qlim[wi] = i4_limb_word<C>(qLs, two_e, wi);
+            } else {
+                for (int wi = tid; wi < 6 * C / 8; wi += kNT)
+                    reinterpret_cast<uint32_t*>(smem + L.ql4)[wi] = i4_limb_word<C>(qLs, two_e, wi);
+            }
+        }
     }
+    if constexpr (kI4Score && C > 32) __syncthreads();  // limbs in shared memory
 
     // [phase] 1
     // ---------------------------------------------------------------- step 2
     // Score one token (local index i) from its label row, store its 16-bit
     // key and count its top byte.
     auto score_token = [&](int i, const uint32_t (&w)[LG::kWords], float ss, float zz) {
-        const float sv = label_score<TKV, LK, C>(w, qreg, qLs, ss, zz, qsum);
+        const float sv = label_score<TKV, LK, C>(w, qreg, qLs, ss, zz, qsum, lim, s_e);
         const uint32_t key = score_key(sv);
         if (!select_all) {
             keys[i] = (uint16_t)(key >> 16);

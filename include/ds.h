@@ -328,7 +328,7 @@ DS_API void ds_sparse_decode_set_cluster(int n);
  *   "scan_prefetch" (0..8, default 2) label scan through registers (when the
  *                   shared-memory ring does not fit): rounds of label rows
  *                   prefetched into L2 ahead.
- *   "i4_ring"       (0 or 1, default 0) 4-bit label rows: when the label ring
+ *   "i4_ring"       (0 or 1, default 1) 4-bit label rows: when the label ring
  *                   and the kept low key bits do not both fit, 1 takes the
  *                   ring (bucket tokens are then re-scored), 0 the low bits. */
 DS_API ds_status ds_sparse_decode_tune(const char* name, int value);
