@@ -126,8 +126,8 @@ bool make_plan(int rows, int G, int s, int d, int c, int topk, bool dense, bool 
             // chunks of 8 tokens, which needs rows of a multiple of 8 tokens
             const int pay = c / 2;
             const bool i4_ring = int4 && s_cap > 0 && s_cap % 8 == 0 && (pay == 4 || pay == 8 || pay % 16 == 0);
-            const int ring = int4 ? (i4_ring ? ds::lab_ring_bytes(pay + 4) : -1)
-                                  : ((c * esz) % 16 == 0 ? ds::lab_ring_bytes(c * esz) : -1);
+            const int ring = int4 ? (i4_ring ? ds::lab_ring_bytes(pay + 4, true) : -1)
+                                  : ((c * esz) % 16 == 0 ? ds::lab_ring_bytes(c * esz, false) : -1);
             // options in order of preference: {bytes, ring, low}; for 4-bit
             // rows, whose re-scoring costs more, the kept low bits come before
             // the ring when only one of them fits

@@ -104,10 +104,13 @@ __host__ __device__ inline int align16(int x) { return (x + 15) & ~15; }
 // (at most 8 * (128 + 2) floats) is later written into its own ring.
 constexpr int kAttStagesF32 = 4;
 // Label-streaming ring (fp labels): stages of one row per thread.
-constexpr int kLabStages = 8;
+// 4-bit rows are short (C/2 + 4 bytes), so their ring is deeper.
+__host__ __device__ constexpr int lab_stages(bool int4) { return int4 ? 12 : 8; }
 // ring bytes for label rows of `label_row_bytes` (a 4-bit row adds its fp16
 // scale and zero, 4 bytes, kept in two arrays of the stage)
-__host__ __device__ constexpr int lab_ring_bytes(int label_row_bytes) { return kLabStages * 256 * label_row_bytes; }
+__host__ __device__ constexpr int lab_ring_bytes(int label_row_bytes, bool int4) {
+    return lab_stages(int4) * 256 * label_row_bytes;
+}
 __host__ __device__ constexpr int att_stage_tokens(int row_bytes, int elem_bytes) {
     return elem_bytes == 2 ? 8 : (row_bytes >= 1024 ? 1 : 1024 / row_bytes);
 }
@@ -128,7 +131,7 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int GT, int D, int C, i
     L.qs = o;     o += align16(GT * D * 4);
     L.qa = o;     o += elem_bytes == 2 ? (D / 16) * 32 * 8 : 0;  // packed bf16 Q fragments
     L.qL = o;     o += align16(C * 4);
-    L.ql4 = o;    o += align16(C * 3);                      // 4-bit scoring: qL as byte limbs
+    L.ql4 = o;    o += align16(C * 3 + 4);                  // 4-bit scoring: qL as byte limbs, 2^-E
     L.idx = o;    o += align16(C * 4);
     L.histA = o;  o += 256 * 4;
     L.histB = o;  o += 256 * 4;
@@ -388,6 +391,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     // zeros of warp w's 32 tokens are 4 + 4 16-byte chunks, copied by lanes
     // 0..7 of that warp (so a __syncwarp makes them visible to its lanes).
     constexpr bool kI4 = LK == kLabelInt4;
+    constexpr int kLabStages = lab_stages(kI4);
     constexpr bool kRingable = kI4 ? (LG::kBytes == 4 || LG::kBytes == 8 || LG::kBytes % 16 == 0)
                                    : LG::kBytes % 16 == 0;
     const bool use_ring = kRingable && need_scores && p.lab_ring;
@@ -453,6 +457,32 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
             for (int e = 0; e < G; ++e) a += qs[e * D + idx_s[j]];
             qLs[j] = a;
         }
+        if constexpr (LK == kLabelInt4 && C <= 32) {
+            // warp 0 already holds qL (lane j has channel j): it forms the
+            // fixed-point limbs for i4_dot once, for every thread to load
+            if (wid == 0) {
+                float qv = 0.f;
+                if (lane < C) {
+                    for (int e = 0; e < G; ++e) qv += qs[e * D + idx_s[lane]];
+                }
+                float qmax = fabsf(qv);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
+                float two_e;
+                const float s_e = i4_scale_exp(qmax, &two_e);
+                const int q = __float2int_rn(__fmul_rn(qv, two_e));
+                // word wi = (k, h, i): byte b is limb k of channel 8i + 2b + h
+                const int wi = lane, k = wi / (2 * (C / 8)), h = (wi / (C / 8)) & 1, i = wi % (C / 8);
+                uint32_t word = 0u;
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const int qc = __shfl_sync(0xffffffffu, q, (8 * i + 2 * b + h) & 31);
+                    word |= ((uint32_t)(qc >> (8 * (k < 3 ? k : 0))) & 255u) << (8 * b);
+                }
+                if (wi < 6 * C / 8) reinterpret_cast<uint32_t*>(smem + L.ql4)[wi] = word;
+                if (lane == 0) reinterpret_cast<float*>(smem + L.ql4)[6 * C / 8] = s_e;
+            }
+        }
     }
     if constexpr (E::kBytes == 2) {
         // tensor-core A fragments of q for the attention phase (see step 3b)
@@ -476,12 +506,43 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
                 srow[j] = x;
                 reinterpret_cast<TKV*>(grow)[j] = x;
             }
-        } else if (lane == 0) {
+        } else {
+            // pack_int4_row's arithmetic with a lane per channel: every lane
+            // forms mn / mx in channel order (as the serial form does), then
+            // lane j divides for channel j and the even lanes pack pairs
             uint16_t* ssz = reinterpret_cast<uint16_t*>(smem + L.app + align16(C * 4));
-            pack_int4_row<TKV>(krow, idx_s, C, smem + L.app, &ssz[0], &ssz[1]);
-            for (int j = 0; j < C / 2; ++j) grow[j] = smem[L.app + j];
-            const_cast<uint16_t*>(lsc)[s - 1] = ssz[0];
-            const_cast<uint16_t*>(lze)[s - 1] = ssz[1];
+            float mn = Elem<TKV>::to_f32(krow[idx_s[0]]), mx = mn;
+            for (int j = 1; j < C; ++j) {
+                const float v = Elem<TKV>::to_f32(krow[idx_s[j]]);
+                mn = fminf(mn, v);
+                mx = fmaxf(mx, v);
+            }
+            const float step = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+            const uint16_t sh = __half_as_ushort(__float2half_rn(step));
+            const uint16_t zh = __half_as_ushort(__float2half_rn(mn));
+            const float sc = fp16_bits_to_f32(sh), z = fp16_bits_to_f32(zh);
+#pragma unroll
+            for (int j0 = 0; j0 < C; j0 += 32) {
+                const int j = j0 + lane;
+                uint32_t code = 0;
+                if (j < C && sc > 0.f) {
+                    float qv = rintf(__fdiv_rn(__fsub_rn(Elem<TKV>::to_f32(krow[idx_s[j]]), z), sc));
+                    qv = fminf(fmaxf(qv, 0.f), 15.f);
+                    code = (uint32_t)qv;
+                }
+                const uint32_t hi = __shfl_down_sync(0xffffffffu, code, 1);
+                if (j < C && !(j & 1)) {
+                    const uint8_t byte = (uint8_t)(code | (hi << 4));
+                    smem[L.app + j / 2] = byte;
+                    grow[j / 2] = byte;
+                }
+            }
+            if (lane == 0) {
+                ssz[0] = sh;
+                ssz[1] = zh;
+                const_cast<uint16_t*>(lsc)[s - 1] = sh;
+                const_cast<uint16_t*>(lze)[s - 1] = zh;
+            }
         }
     }
     __syncthreads();
@@ -525,14 +586,17 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         }
         for (int j = 0; j < C; ++j) qsum += qLs[j];
         if constexpr (kI4Score) {
-            float qmax = 0.f;
-            for (int j = 0; j < C; ++j) qmax = fmaxf(qmax, fabsf(qLs[j]));
-            float two_e;
-            s_e = i4_scale_exp(qmax, &two_e);
             if constexpr (C <= 32) {
+                // formed by warp 0 before the barrier above
+                const uint32_t* lw = reinterpret_cast<const uint32_t*>(smem + L.ql4);
 #pragma unroll
-                for (int wi = 0; wi < 6 * C / 8; ++wi) qlim[wi] = i4_limb_word<C>(qLs, two_e, wi);
+                for (int wi = 0; wi < 6 * C / 8; ++wi) qlim[wi] = lw[wi];
+                s_e = reinterpret_cast<const float*>(smem + L.ql4)[6 * C / 8];
             } else {
+                float qmax = 0.f;
+                for (int j = 0; j < C; ++j) qmax = fmaxf(qmax, fabsf(qLs[j]));
+                float two_e;
+                s_e = i4_scale_exp(qmax, &two_e);
                 for (int wi = tid; wi < 6 * C / 8; wi += kNT)
                     reinterpret_cast<uint32_t*>(smem + L.ql4)[wi] = i4_limb_word<C>(qLs, two_e, wi);
             }
