@@ -75,7 +75,7 @@ constexpr int kMaxSmem = 227 * 1024;
 constexpr int kCtasPerSm = 2;  // __launch_bounds__(256, 2) -> <= 128 registers
 
 struct Plan {
-    int N, chunk, lay_chunk, per, smem, att_stages, lab_ring, keep_low;
+    int N, chunk, lay_chunk, per, smem, att_stages, lab_ring, keep_low, sel_off;
 };
 
 // Two CTAs of 256 threads per SM: each may use up to (228 KiB - 2 KiB) / 2.
@@ -92,7 +92,7 @@ bool make_plan(int rows, int G, int s, int d, int c, int topk, bool dense, bool 
     const int GT = group_tier(G);
     const bool select_all = dense || topk >= s;
     const int k_eff = topk < s ? topk : s;
-    Plan best{0, 0, 0, 0, 0, 0, 0, 0};
+    Plan best{0, 0, 0, 0, 0, 0, 0, 0, 0};
     for (int N = 1; N <= 16; N *= 2) {
         Plan p;
         p.N = N;
@@ -100,11 +100,14 @@ bool make_plan(int rows, int G, int s, int d, int c, int topk, bool dense, bool 
         if (p.chunk > ds::kMaxChunk) continue;
         p.lay_chunk = dense ? 0 : p.chunk;
         p.per = select_all ? 0 : (k_eff + N - 1) / N;
-        // bf16 K/V: 3 attention stages per warp when two CTAs still fit per SM, else 2
+        // bf16 K/V: 3 attention stages per warp when two CTAs still fit per SM
+        // (with the selection's needs below), else 2
         p.att_stages = esz == 2 ? 3 : ds::kAttStagesF32;
         p.smem = ds::decode_smem_layout(GT, d, c, p.lay_chunk, p.per, esz, p.att_stages).total;
-        if (esz == 2 && p.smem > kSmemFor2) {
-            p.att_stages = 2;
+        const int sel_need = dense ? 0 : ds::align16(p.lay_chunk * 2) + ds::sel_scratch_bytes(p.lay_chunk);
+        if (esz == 2) {
+            const ds::DecodeSmem L3 = ds::decode_smem_layout(GT, d, c, p.lay_chunk, p.per, esz, 3, sel_need);
+            if (L3.total > kSmemFor2) p.att_stages = 2;
             p.smem = ds::decode_smem_layout(GT, d, c, p.lay_chunk, p.per, esz, p.att_stages).total;
         }
         if (p.smem > kMaxSmem) continue;
@@ -139,14 +142,22 @@ bool make_plan(int rows, int G, int s, int d, int c, int topk, bool dense, bool 
                 {2 * keys, 0, 1},
                 {ring >= 0 ? keys + ring : -1, 1, 0},
             };
+            // the selection scratch sits behind the keys (and kept low bits),
+            // over the label ring, which is dead by then
+            const int scratch = ds::sel_scratch_bytes(p.lay_chunk);
+            int used = keys + scratch;
             for (const Opt& o : opts) {
-                if (o.need < 0 || o.need > cap) continue;
+                if (o.need < 0) continue;
+                const int need_o = o.need > (o.low ? 2 : 1) * keys + scratch ? o.need : (o.low ? 2 : 1) * keys + scratch;
+                if (need_o > cap) continue;
                 p.lab_ring = o.ring;
                 p.keep_low = o.low;
-                if (o.need > region_att)
-                    p.smem = ds::decode_smem_layout(GT, d, c, p.lay_chunk, p.per, esz, p.att_stages, o.need).total;
+                used = need_o;
                 break;
             }
+            p.sel_off = keys * (p.keep_low ? 2 : 1);
+            if (used > region_att)
+                p.smem = ds::decode_smem_layout(GT, d, c, p.lay_chunk, p.per, esz, p.att_stages, used).total;
         }
         if (forced) {
             if (N == forced) { *out = p; return true; }
@@ -613,6 +624,7 @@ ds_status sparse_decode_impl(const void* q, const void* k, const void* v, ds_dty
     p.out_bf16 = out_dt == DS_BF16;
     p.dense = 0;
     p.scan_prefetch = g_scan_prefetch.load();
+    p.sel_off = pl.sel_off;
     return launch_decode(kern, p, rows, pl, stream);
 }
 

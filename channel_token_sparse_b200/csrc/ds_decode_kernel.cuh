@@ -77,6 +77,10 @@ struct DecodeParams {
     const void* v_new;
     // label rounds pulled into L2 ahead of the register-path scan (0: none)
     int scan_prefetch;
+    // byte offset in the region of the selection scratch (bucket flags, mask
+    // cache, bucket list): behind the 16-bit keys and kept low bits, over the
+    // label ring, which is dead by the time the selection starts
+    int sel_off;
 };
 
 // Row (in units of d elements) of token t of (b, g) in the K/V caches, dense
@@ -91,10 +95,15 @@ __device__ __forceinline__ size_t kv_row_of(const DecodeParams& p, int b, int g,
 
 // Shared-memory carve-up (bytes), identical on host and device.
 struct DecodeSmem {
-    int qs, qa, qL, ql4, idx, histA, histB, ctl, scan, cm, cl, co, bits, mcache, blist, app, sel, region, total;
+    int qs, qa, qL, ql4, idx, histA, histB, ctl, scan, cm, cl, co, krow, app, sel, region, total;
 };
 
 __host__ __device__ inline int align16(int x) { return (x + 15) & ~15; }
+
+// Selection scratch in the region (see DecodeParams::sel_off): bucket flags
+// (a byte per 8 tokens), the per-group selected / tie mask cache (2 bytes per
+// 8 tokens) and the bucket list (kBucketCap words).
+__host__ __device__ inline int sel_scratch_bytes(int chunk);
 
 // Attention-phase staging: each warp owns a ring of shared-memory stages; a
 // stage holds the K rows then the V rows of att_stage_tokens() tokens. With
@@ -104,8 +113,9 @@ __host__ __device__ inline int align16(int x) { return (x + 15) & ~15; }
 // (at most 8 * (128 + 2) floats) is later written into its own ring.
 constexpr int kAttStagesF32 = 4;
 // Label-streaming ring (fp labels): stages of one row per thread.
-// 4-bit rows are short (C/2 + 4 bytes), so their ring is deeper.
-__host__ __device__ constexpr int lab_stages(bool int4) { return int4 ? 12 : 8; }
+// Stages of the label ring (8 for both kinds: a 12-stage ring for the short
+// 4-bit rows was measured no faster).
+__host__ __device__ constexpr int lab_stages(bool) { return 8; }
 // ring bytes for label rows of `label_row_bytes` (a 4-bit row adds its fp16
 // scale and zero, 4 bytes, kept in two arrays of the stage)
 __host__ __device__ constexpr int lab_ring_bytes(int label_row_bytes, bool int4) {
@@ -121,6 +131,9 @@ __host__ __device__ constexpr int att_ring_bytes(int row_bytes, int elem_bytes, 
 // pass (a CTA whose bucket is larger falls back to sweeping its keys).
 constexpr int kBucketCap = 1024;
 constexpr int kMaxCluster = 16;  // CTAs per row at most (portable 8, non-portable 16)
+__host__ __device__ inline int sel_scratch_bytes(int chunk) {
+    return align16(chunk / 8) + align16(chunk / 8 * 2) + kBucketCap * 4;
+}
 
 // region_min: room the selection phase wants for the label ring and the
 // low key bits beyond the keys and the attention ring (host plans only).
@@ -140,9 +153,7 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int GT, int D, int C, i
     L.cm = o;     o += align16(kMaxCluster * GT * 4);        // cluster merge: (m, l) of every CTA
     L.cl = o;     o += align16(kMaxCluster * GT * 4);
     L.co = o;     o += align16((GT * D + kMaxCluster) * 4);  // cluster merge: partial o received
-    L.bits = o;   o += align16(chunk / 8);
-    L.mcache = o; o += align16(chunk / 8 * 2);  // per key group: selected / tie masks
-    L.blist = o;  o += chunk > 0 ? kBucketCap * 4 : 0;
+    L.krow = o;   o += align16(D * elem_bytes);            // the appended token's key row
     L.app = o;    o += align16(C * 4) + 16;  // appended token's label row (+ fp16 scale, zero)
     L.sel = o;    o += align16(per * 4);
     L.region = o;
@@ -317,9 +328,9 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     float* cm = reinterpret_cast<float*>(smem + L.cm);
     float* cl = reinterpret_cast<float*>(smem + L.cl);
     float* co = reinterpret_cast<float*>(smem + L.co);
-    uint8_t* bits8 = smem + L.bits;                     // bucket flags, one byte per 8 tokens
-    uint16_t* mcache = reinterpret_cast<uint16_t*>(smem + L.mcache);
-    uint32_t* blist = reinterpret_cast<uint32_t*>(smem + L.blist);
+    uint8_t* bits8 = smem + L.region + p.sel_off;       // bucket flags, one byte per 8 tokens
+    uint16_t* mcache = reinterpret_cast<uint16_t*>(bits8 + align16(p.lay_chunk / 8));
+    uint32_t* blist = reinterpret_cast<uint32_t*>(bits8 + align16(p.lay_chunk / 8) + align16(p.lay_chunk / 8 * 2));
     int* sel_list = reinterpret_cast<int*>(smem + L.sel);
     uint16_t* keys = reinterpret_cast<uint16_t*>(smem + L.region);
 
@@ -432,9 +443,8 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
 #pragma unroll
     for (int e = 0; e < kQPer; ++e)
         if (tid + kNT * e < G * D) qs[tid + kNT * e] = qv[e];
-    // the newest token's key row is staged in the bucket list (unused until
-    // the selection; a decode step always has one)
-    uint8_t* krow_s = reinterpret_cast<uint8_t*>(blist);
+    // the newest token's key row is staged in shared memory
+    uint8_t* krow_s = smem + L.krow;
     if (app_i >= 0 && tid < kKRowVecs) {
         reinterpret_cast<uint4*>(krow_s)[tid] = kv_app;
         if (p.k_new) {  // the new token's K/V rows into the caches (read back by the attention)
