@@ -156,6 +156,16 @@ bool make_plan(int rows, int G, int s, int d, int c, int topk, bool dense, bool 
                 break;
             }
             p.sel_off = keys * (p.keep_low ? 2 : 1);
+            // without the label ring the scan's register loads live in L1,
+            // which shares the SM's storage with shared memory: such rows
+            // keep 2 attention stages (3 cost the 256K layer 11 us)
+            if (!p.lab_ring && p.att_stages == 3 && esz == 2) {
+                p.att_stages = 2;
+                const ds::DecodeSmem L2s = ds::decode_smem_layout(GT, d, c, p.lay_chunk, p.per, esz, 2);
+                p.smem = L2s.total;
+                if (used > L2s.total - L2s.region)
+                    p.smem = ds::decode_smem_layout(GT, d, c, p.lay_chunk, p.per, esz, 2, used).total;
+            }
             if (used > region_att)
                 p.smem = ds::decode_smem_layout(GT, d, c, p.lay_chunk, p.per, esz, p.att_stages, used).total;
         }

@@ -437,7 +437,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     };
     if (use_ring) {
 #pragma unroll 1
-        for (int j = 0; j < kLabStages - 1; ++j) { issue(j); cp_async_commit(); }
+        for (int j = 0; j < kLabStages - 2; ++j) { issue(j); cp_async_commit(); }
     }
 
 #pragma unroll
@@ -618,8 +618,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     // ---------------------------------------------------------------- step 2
     // Score one token (local index i) from its label row, store its 16-bit
     // key and count its top byte.
-    auto score_token = [&](int i, const uint32_t (&w)[LG::kWords], float ss, float zz) {
-        const float sv = label_score<TKV, LK, C>(w, qreg, qLs, ss, zz, qsum, lim, s_e);
+    auto record_token = [&](int i, float sv) {
         const uint32_t key = score_key(sv);
         if (!select_all) {
             keys[i] = (uint16_t)(key >> 16);
@@ -628,31 +627,44 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         }
         if (p.score_out) p.score_out[(size_t)row * p.s + t0 + i] = sv;
     };
+    auto score_token = [&](int i, const uint32_t (&w)[LG::kWords], float ss, float zz) {
+        record_token(i, label_score<TKV, LK, C>(w, qreg, qLs, ss, zz, qsum, lim, s_e));
+    };
     if (use_ring) {
+        // two stages per iteration: each thread scores two tokens (j and
+        // j + 1 stages apart) whose arithmetic chains are independent
+        auto stage_row = [&](int j, int i, uint32_t (&w)[LG::kWords], float& ss, float& zz) {
+            const uint8_t* stg = lring + (j % kLabStages) * kStage;
+            if (i == app_i) {
+                lds_row<LG::kBytes>(w, app_row);
+                if constexpr (kI4) { ss = fp16_bits_to_f32(app_sz[0]); zz = fp16_bits_to_f32(app_sz[1]); }
+            } else {
+                lds_row<LG::kBytes>(w, stg + tid * kSlot);
+                if constexpr (kI4) {
+                    ss = fp16_bits_to_f32(reinterpret_cast<const uint16_t*>(stg + kNT * kSlot)[tid]);
+                    zz = fp16_bits_to_f32(reinterpret_cast<const uint16_t*>(stg + kNT * kSlot + kNT * 2)[tid]);
+                }
+            }
+        };
 #pragma unroll 1
-        for (int j = 0; j < nst; ++j) {
-            if constexpr (kI4) __syncwarp();   // every lane is done with the slot refilled next
+        for (int j = 0; j < nst; j += 2) {
+            if constexpr (kI4) __syncwarp();   // every lane is done with the slots refilled next
+            issue(j + kLabStages - 2);
+            cp_async_commit();
             issue(j + kLabStages - 1);
             cp_async_commit();
-            cp_async_wait<kLabStages - 1>();
+            cp_async_wait<kLabStages - 2>();   // stages j and j + 1 have landed
             if constexpr (kI4) __syncwarp();   // the warp's scale / zero chunks
-            const int i = j * kNT + tid;
-            if (i < n_loc) {
-                uint32_t w[LG::kWords];
-                const uint8_t* stg = lring + (j % kLabStages) * kStage;
-                float ss = 0.f, zz = 0.f;
-                if (i == app_i) {
-                    lds_row<LG::kBytes>(w, app_row);
-                    if constexpr (kI4) { ss = fp16_bits_to_f32(app_sz[0]); zz = fp16_bits_to_f32(app_sz[1]); }
-                } else {
-                    lds_row<LG::kBytes>(w, stg + tid * kSlot);
-                    if constexpr (kI4) {
-                        ss = fp16_bits_to_f32(reinterpret_cast<const uint16_t*>(stg + kNT * kSlot)[tid]);
-                        zz = fp16_bits_to_f32(reinterpret_cast<const uint16_t*>(stg + kNT * kSlot + kNT * 2)[tid]);
-                    }
-                }
-                score_token(i, w, ss, zz);
-            }
+            const int i0 = j * kNT + tid, i1 = i0 + kNT;
+            uint32_t w0[LG::kWords], w1[LG::kWords];
+            float ss0 = 0.f, zz0 = 0.f, ss1 = 0.f, zz1 = 0.f;
+            stage_row(j, i0, w0, ss0, zz0);
+            stage_row(j + 1, i1, w1, ss1, zz1);
+            // rows past the chunk hold stale ring bytes: scored, not recorded
+            const float sv0 = label_score<TKV, LK, C>(w0, qreg, qLs, ss0, zz0, qsum, lim, s_e);
+            const float sv1 = label_score<TKV, LK, C>(w1, qreg, qLs, ss1, zz1, qsum, lim, s_e);
+            if (i0 < n_loc) record_token(i0, sv0);
+            if (i1 < n_loc) record_token(i1, sv1);
         }
         cp_async_wait<0>();
     } else if (need_scores) {
