@@ -378,6 +378,52 @@ def decode_step_kv(q, k_new, v_new, k, v, label, idx, s: int, topk: int, lscale=
     return out
 
 
+class PreparedDecodeStepKV:
+    """decode_step_kv with every argument checked and converted once.
+
+    A serving loop decodes token after token into the same caches, label
+    cache and (pinned host or device) buffers; only their contents and the
+    token count change. Preparing the call keeps the per-step host cost to
+    one C-ABI call: ``step()`` enqueues one step (ds_decode_step_kv) on the
+    stream that was current at preparation (or `stream`), and
+    ``step.set_length(s)`` moves to another token count."""
+
+    _S_ARG = 14  # position of `s` in the ds_decode_step_kv argument list
+
+    def __init__(self, q, k_new, v_new, k, v, label, idx, s: int, topk: int, lscale=None, lzero=None,
+                 out=None, out_dtype=None, sm_scale: float = 0.0, stream=None):
+        torch = _torch()
+        _need_cuda_or_pinned(k, v, q, k_new, v_new)
+        _need_cuda(label, idx, lscale, lzero)
+        b, hq, d = q.shape
+        _, hkv, s_cap, _ = k.shape
+        c = idx.shape[1]
+        kdt = _kv_dtype(k)
+        if k_new.dtype != k.dtype or v_new.dtype != v.dtype:
+            raise TypeError("k_new / v_new must have the caches' dtype")
+        if out is None:
+            out = torch.empty((b, hq, d), dtype=out_dtype or torch.float32, device=label.device)
+        _need_cuda_or_pinned(out)
+        odt = DS_F32 if out.dtype == torch.float32 else DS_BF16
+        self.out = out
+        self._keep = (q, k_new, v_new, k, v, label, idx, lscale, lzero, out)  # keep the memory alive
+        self._args = [_ptr_kv(q), _ptr_kv(k_new), _ptr_kv(v_new), _ptr_kv(k), _ptr_kv(v), kdt, _ptr(label),
+                      _label_args(label, lscale, lzero, kdt), _ptr(lscale), _ptr(lzero), _ptr(idx), b, hq, hkv,
+                      int(s), s_cap, d, c, int(topk), float(sm_scale), _ptr_kv(out), odt, None, None,
+                      _stream(stream)]
+        assert self._args[self._S_ARG - 1] == hkv and self._args[self._S_ARG + 1] == s_cap  # layout check
+        self._fn = lib().ds_decode_step_kv
+
+    def set_length(self, s: int) -> None:
+        self._args[self._S_ARG] = int(s)
+
+    def __call__(self):
+        st = self._fn(*self._args)
+        if st != DS_OK:
+            raise DSError(st, last_error())
+        return self.out
+
+
 def decode_step_varlen(q, k, v, label, idx, seq_lens, s_max: int, topk: int, lscale=None, lzero=None, out=None,
                        out_dtype=None, sm_scale: float = 0.0, sel_out=None, score_out=None,
                        sparse_threshold: int = 0, fallback: int = DS_FALLBACK_PER_ENTRY, stream=None):

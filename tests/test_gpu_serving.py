@@ -486,3 +486,35 @@ def test_decode_step_kv_from_host_buffers(kv, label, cluster, out_dtype):
     assert torch.equal(oh, od.cpu())
     with pytest.raises(ValueError):  # pageable host memory is refused
         ds.decode_step_kv(qd.cpu(), k_new, v_new, k1, v1, lab, idxd, s, topk, lscale=sc, lzero=ze, out=od)
+
+
+def test_prepared_decode_step_equals_call():
+    """PreparedDecodeStepKV (arguments bound once) gives the bits of
+    decode_step_kv, from host buffers, and follows set_length."""
+    b, hq, hkv, d, c, s, topk = 2, 8, 4, 128, 16, 2500, 128
+    wl = synth.custom(b=b, hq=hq, hkv=hkv, d=d, s=s, c=c, topk=topk, kv_dtype="bf16", label_dtype="bf16",
+                      n_outlier=16, outlier_scale=6.0, index=88)
+    di = synth.decode_inputs(wl, s_cap=s + 8)
+    idxd = torch.from_numpy(_idx_random(wl, 16)).cuda()
+    qd, kd, vd = (to_dev(x, "bf16") for x in (di.q, di.k, di.v))
+    outs = []
+    for length in (s, s - 300):
+        k_new, v_new = kd[:, :, length - 1].clone(), vd[:, :, length - 1].clone()
+        runs = []
+        for mode in ("call", "prepared"):
+            k1, v1 = kd.clone(), vd.clone()
+            lab, _, _ = _label_alloc(kd, wl)
+            ds.build_label_cache(kd, idxd, length - 1, lab)
+            qh, knh, vnh = (t.cpu().pin_memory() for t in (qd, k_new, v_new))
+            oh = torch.zeros((b, hq, d), dtype=torch.bfloat16).pin_memory()
+            if mode == "call":
+                ds.decode_step_kv(qh, knh, vnh, k1, v1, lab, idxd, length, topk, out=oh)
+            else:
+                step = ds.PreparedDecodeStepKV(qh, knh, vnh, k1, v1, lab, idxd, s, topk, out=oh)
+                step.set_length(length)
+                step()
+            torch.cuda.synchronize()
+            runs.append((oh.clone(), lab.clone()))
+        assert torch.equal(runs[0][0], runs[1][0]) and torch.equal(runs[0][1], runs[1][1])
+        outs.append(runs[0][0])
+    assert not torch.equal(outs[0], outs[1])
