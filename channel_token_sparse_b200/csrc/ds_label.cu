@@ -77,20 +77,92 @@ __global__ void __launch_bounds__(kLabNT) ds_label_kernel(const TKV* __restrict_
 // in), so the next blocks' reads are in flight while the current one is
 // gathered or packed. Same results as ds_label_kernel.
 constexpr int kBulkStage = 16384;  // bytes of key rows per stage
-constexpr int kBulkStages = 4;
+constexpr int kBulkStages = 6;
 constexpr int kBulkNT = 256;
 // packing threads per token (4-bit): each takes c / kPackLanes channels
 constexpr int kPackLanes = 4;
 
 __host__ __device__ constexpr int bulk_smem_bytes() { return kBulkStages * kBulkStage + kBulkStages * 8; }
 
-// CI: the channel count, fixed at compile time for 4-bit rows (each lane's
-// CI / kPackLanes channel indices then stay in registers); 0 for fp rows.
+// A CTA's items are blockIdx.x, blockIdx.x + gridDim.x, ... in (row, block)
+// order; the cursor steps to the next one with adds and one carry instead of
+// a division per item.
+struct ItemCursor {
+    int row, blk, g;            // current item: row = b * hkv + g, block of the row
+    int rstep, bstep, gstep;    // gridDim.x = rstep * nblk + bstep; gstep = rstep % hkv
+    int nblk, hkv;
+    __device__ __forceinline__ void init(int first, int grid, int nblk_, int hkv_) {
+        nblk = nblk_;
+        hkv = hkv_;
+        row = first / nblk;
+        blk = first - row * nblk;
+        g = row % hkv;
+        rstep = grid / nblk;
+        bstep = grid - rstep * nblk;
+        gstep = rstep % hkv;
+    }
+    __device__ __forceinline__ void next() {
+        blk += bstep;
+        row += rstep;
+        g += gstep;
+        if (blk >= nblk) {
+            blk -= nblk;
+            ++row;
+            ++g;
+        }
+        if (g >= hkv) g -= hkv;
+    }
+};
+
+// 4-bit codes of n values a_e = x_e - zero: the quotient a_e / scale is
+// formed with the rounded reciprocal, and only where it lies within 1e-5 of a
+// half-integer (where the two could round differently) is it recomputed with
+// the IEEE division; rint (half to even) then clamp to [0, 15], which
+// __float2int_rn followed by an integer clamp gives for every input (NaN
+// converts to 0). The codes equal those of int4_code.
+template <int N>
+__device__ __forceinline__ void int4_codes(const float (&a)[N], float sc, float rcp_sc, uint32_t (&code)[N]) {
+    float q[N];
+    uint32_t near = 0u;
+#pragma unroll
+    for (int e = 0; e < N; ++e) {
+        q[e] = __fmul_rn(a[e], rcp_sc);
+        if (fabsf(q[e] - floorf(q[e]) - 0.5f) <= 1e-5f) near |= 1u << e;
+    }
+    if (near) {
+#pragma unroll
+        for (int e = 0; e < N; ++e)
+            if ((near >> e) & 1u) q[e] = __fdiv_rn(a[e], sc);
+    }
+#pragma unroll
+    for (int e = 0; e < N; ++e) code[e] = sc > 0.f ? (uint32_t)min(max(__float2int_rn(q[e]), 0), 15) : 0u;
+}
+
+// Pick element (p - r) & 3 of a: the value a rotated thread read for output
+// position p.
+__device__ __forceinline__ uint32_t pick_rot(const uint32_t (&a)[4], int p, int r) {
+    const int e = (p - r) & 3;
+    return e == 0 ? a[0] : (e == 1 ? a[1] : (e == 2 ? a[2] : a[3]));
+}
+
+// CI: the channel count, fixed at compile time, so the per-thread channel
+// lists stay in registers and the token / channel arithmetic is shifts.
+//
+// fp rows: a thread writes 4 consecutive label elements of one token (one
+// 8-byte store for bf16, 16 bytes for fp32). The tokens a warp covers lie a
+// multiple of 128 bytes apart in the ring, so one channel of each of them
+// falls in the same bank: each thread reads its 4 channels rotated by its
+// token index (t & 3) and rotates the values back, so at each step the
+// warp's tokens read different channels.
+// 4-bit rows: kPackLanes threads per token with CI / kPackLanes channels
+// each, rotated the same way by the token's slot in the warp; the arithmetic
+// is that of pack_int4_row, with mn / mx combined over the lanes (fminf /
+// fmaxf do not depend on the order).
 template <typename TKV, int LK, int D, int CI>
 __global__ void __launch_bounds__(kBulkNT, 2) ds_label_bulk_kernel(const TKV* __restrict__ k,
                                                                   const int32_t* __restrict__ idx, int hkv,
-                                                                  int t_begin, int t_end, int s_cap, int c,
-                                                                  int rows, uint8_t* __restrict__ label,
+                                                                  int t_begin, int t_end, int s_cap, int rows,
+                                                                  uint8_t* __restrict__ label,
                                                                   uint16_t* __restrict__ lscale,
                                                                   uint16_t* __restrict__ lzero,
                                                                   unsigned int* __restrict__ err) {
@@ -101,69 +173,98 @@ __global__ void __launch_bounds__(kBulkNT, 2) ds_label_bulk_kernel(const TKV* __
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + kBulkStages * kBulkStage);
     const int tid = threadIdx.x;
     const int nblk = (t_end - t_begin + kTok - 1) / kTok;  // blocks per row
-    const long long items = (long long)rows * nblk;
+    const int items = rows * nblk;                          // below 2^30 (checked by the host)
     if (tid == 0) {
         for (int i = 0; i < kBulkStages; ++i) mbar_init(&full[i], 1);
         fence_mbar_init();
     }
     __syncthreads();
-    auto issue = [&](long long it, int slot) {
-        const int row = (int)(it / nblk), blk = (int)(it - (long long)row * nblk);
-        const int tb = t_begin + blk * kTok;
+    // producer (thread 0): the item kBulkStages ahead of the consumer's
+    ItemCursor pc{};
+    int pit = blockIdx.x;
+    auto issue = [&](int slot) {
+        const int tb = t_begin + pc.blk * kTok;
         const int nt = min(kTok, t_end - tb);
         const uint32_t bytes = (uint32_t)(nt * kRowBytes);
         mbar_arrive_expect_tx(&full[slot], bytes);
-        bulk_g2s(sm + slot * kBulkStage, k + ((size_t)row * s_cap + tb) * D, bytes, &full[slot]);
+        bulk_g2s(sm + slot * kBulkStage, k + ((size_t)pc.row * s_cap + tb) * D, bytes, &full[slot]);
+        pit += gridDim.x;
+        pc.next();
     };
-    if (tid == 0)
-        for (int i = 0; i < kBulkStages; ++i) {
-            const long long it = blockIdx.x + (long long)i * gridDim.x;
-            if (it < items) issue(it, i);
-        }
-    constexpr int kPer = CI / kPackLanes > 0 ? CI / kPackLanes : 1;  // 4-bit channels per lane
+    if (tid == 0) {
+        pc.init(blockIdx.x, gridDim.x, nblk, hkv);
+        for (int i = 0; i < kBulkStages && pit < items; ++i) issue(i);
+    }
+
+    constexpr int kG = CI / 4;                  // fp: 4-element groups per label row
+    const int fq = tid % kG, frot = (tid / kG) & 3;
+    // fp, bf16: byte selectors that rotate 4 packed 16-bit values left by frot
+    const uint32_t sel_lo = ((0u - 2 * frot) & 7) | (((1u - 2 * frot) & 7) << 4) | (((2u - 2 * frot) & 7) << 8) |
+                            (((3u - 2 * frot) & 7) << 12);
+    const uint32_t sel_hi = ((4u - 2 * frot) & 7) | (((5u - 2 * frot) & 7) << 4) | (((6u - 2 * frot) & 7) << 8) |
+                            (((7u - 2 * frot) & 7) << 12);
+    constexpr int kPer = CI / kPackLanes > 0 ? CI / kPackLanes : 1;  // 4-bit: channels per lane
+    constexpr bool kRot = kPer <= 16;  // a lane's nibbles fit one 64-bit word
+    const int q4 = tid % kPackLanes;
+    const int rot = kRot ? (tid / kPackLanes) % kPer : 0;
+    constexpr int kOff = LK == 0 ? 4 : kPer;
+    int off[kOff];  // this thread's channels, in its rotated order
     int g_cur = -1;
-    int my_idx[kPer];  // 4-bit: this thread's channels
-    int fp_idx = 0;    // fp: this thread's channel (tid % c)
-    int j = 0;
-    for (long long it = blockIdx.x; it < items; it += gridDim.x, ++j) {
+    ItemCursor cc;
+    cc.init(blockIdx.x, gridDim.x, nblk, hkv);
+    for (int it = blockIdx.x, j = 0; it < items; it += gridDim.x, ++j, cc.next()) {
         const int slot = j % kBulkStages;
-        const int row = (int)(it / nblk), blk = (int)(it - (long long)row * nblk);
-        const int g = row % hkv;
-        const int tb = t_begin + blk * kTok;
+        const int tb = t_begin + cc.blk * kTok;
         const int nt = min(kTok, t_end - tb);
-        const size_t tok0 = (size_t)row * s_cap + tb;
-        if (g != g_cur) {
-            g_cur = g;
-            if constexpr (LK == 0) {
-                fp_idx = min(max(__ldg(idx + (size_t)g * c + tid % c), 0), D - 1);
-            } else {
-                const int q = tid % kPackLanes;
+        const size_t tok0 = (size_t)cc.row * s_cap + tb;
+        if (cc.g != g_cur) {
+            g_cur = cc.g;
+            const int32_t* ig = idx + (size_t)g_cur * CI;
 #pragma unroll
-                for (int e = 0; e < kPer; ++e)
-                    my_idx[e] = min(max(__ldg(idx + (size_t)g * CI + q * kPer + e), 0), D - 1);
+            for (int e = 0; e < kOff; ++e) {
+                const int ch = LK == 0 ? 4 * fq + ((e + frot) & 3) : q4 * kPer + ((e + rot) % kPer);
+                off[e] = min(max(__ldg(ig + ch), 0), D - 1);
             }
         }
         const bool ok = mbar_wait_bounded(&full[slot], (uint32_t)((j / kBulkStages) & 1), err, 1);
-        const TKV* rows_s = reinterpret_cast<const TKV*>(sm + slot * kBulkStage);
         if (ok) {
             if constexpr (LK == 0) {
-                // thread tid always handles channel tid % c (c divides the CTA size)
-                TKV* out = reinterpret_cast<TKV*>(label) + tok0 * c;
-                for (int e = tid; e < nt * c; e += kBulkNT) out[e] = rows_s[(e / c) * D + fp_idx];
+                if constexpr (E::kBytes == 2) {
+                    const uint16_t* rs = reinterpret_cast<const uint16_t*>(sm + slot * kBulkStage);
+                    uint16_t* out = reinterpret_cast<uint16_t*>(label) + tok0 * CI + 4 * fq;
+                    for (int t = tid / kG; t < nt; t += kBulkNT / kG) {
+                        const uint16_t* x = rs + t * D;
+                        const uint32_t p01 = __byte_perm(x[off[0]], x[off[1]], 0x5410);
+                        const uint32_t p23 = __byte_perm(x[off[2]], x[off[3]], 0x5410);
+                        uint2 w;
+                        w.x = __byte_perm(p01, p23, sel_lo);
+                        w.y = __byte_perm(p01, p23, sel_hi);
+                        *reinterpret_cast<uint2*>(out + (size_t)t * CI) = w;
+                    }
+                } else {
+                    const uint32_t* rs = reinterpret_cast<const uint32_t*>(sm + slot * kBulkStage);
+                    uint32_t* out = reinterpret_cast<uint32_t*>(label) + tok0 * CI + 4 * fq;
+                    for (int t = tid / kG; t < nt; t += kBulkNT / kG) {
+                        const uint32_t* x = rs + t * D;
+                        const uint32_t a[4] = {x[off[0]], x[off[1]], x[off[2]], x[off[3]]};
+                        *reinterpret_cast<uint4*>(out + (size_t)t * CI) =
+                            make_uint4(pick_rot(a, 0, frot), pick_rot(a, 1, frot), pick_rot(a, 2, frot),
+                                       pick_rot(a, 3, frot));
+                    }
+                }
             } else {
-                // kPackLanes threads per token, c / kPackLanes channels each:
-                // the arithmetic of pack_int4_row, with mn / mx combined over
-                // the lanes (fminf / fmaxf do not depend on the order)
-                const int q = tid % kPackLanes;
+                const TKV* rows_s = reinterpret_cast<const TKV*>(sm + slot * kBulkStage);
                 for (int t = tid / kPackLanes; t < ((nt + 7) & ~7); t += kBulkNT / kPackLanes) {
                     const bool live = t < nt;
                     const TKV* x = rows_s + (size_t)(live ? t : 0) * D;
-                    float mn = E::to_f32(x[my_idx[0]]), mx = mn;
+                    float v[kPer];
+#pragma unroll
+                    for (int e = 0; e < kPer; ++e) v[e] = E::to_f32(x[off[e]]);
+                    float mn = v[0], mx = v[0];
 #pragma unroll
                     for (int e = 1; e < kPer; ++e) {
-                        const float v = E::to_f32(x[my_idx[e]]);
-                        mn = fminf(mn, v);
-                        mx = fmaxf(mx, v);
+                        mn = fminf(mn, v[e]);
+                        mx = fmaxf(mx, v[e]);
                     }
 #pragma unroll
                     for (int o = 1; o < kPackLanes; o <<= 1) {
@@ -176,16 +277,29 @@ __global__ void __launch_bounds__(kBulkNT, 2) ds_label_bulk_kernel(const TKV* __
                     const float sc = fp16_bits_to_f32(sh), z = fp16_bits_to_f32(zh);
                     const float rsc = sc > 0.f ? __frcp_rn(sc) : 0.f;
                     if (live) {
-                        uint8_t* dst = label + (tok0 + t) * (size_t)(CI / 2) + q * kPer / 2;
+                        float a[kPer];
 #pragma unroll
-                        for (int e = 0; e < kPer; e += 2) {
-                            uint32_t nib[2];
+                        for (int e = 0; e < kPer; ++e) a[e] = __fsub_rn(v[e], z);
+                        uint32_t code[kPer];
+                        int4_codes<kPer>(a, sc, rsc, code);
+                        // channel q4 * kPer + e of the row is nibble e of this
+                        // lane's kPer / 2 bytes (low nibble first)
+                        uint8_t* dst = label + (tok0 + t) * (size_t)(CI / 2) + q4 * kPer / 2;
+                        if constexpr (kRot) {
+                            uint64_t w = 0;
 #pragma unroll
-                            for (int h = 0; h < 2; ++h)
-                                nib[h] = sc > 0.f ? int4_code(E::to_f32(x[my_idx[e + h]]), z, sc, rsc) : 0u;
-                            dst[e / 2] = (uint8_t)(nib[0] | (nib[1] << 4));
+                            for (int e = 0; e < kPer; ++e) w |= (uint64_t)code[e] << (4 * ((e + rot) % kPer));
+                            // dst is kPer / 2-byte aligned: label is 16-byte
+                            // aligned and rows are 2 * kPer bytes long
+                            if constexpr (kPer == 2) *dst = (uint8_t)w;
+                            else if constexpr (kPer == 4) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)w;
+                            else if constexpr (kPer == 8) *reinterpret_cast<uint32_t*>(dst) = (uint32_t)w;
+                            else *reinterpret_cast<uint64_t*>(dst) = w;
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < kPer; e += 2) dst[e / 2] = (uint8_t)(code[e] | (code[e + 1] << 4));
                         }
-                        if (q == 0) {
+                        if (q4 == 0) {
                             lscale[tok0 + t] = sh;
                             lzero[tok0 + t] = zh;
                         }
@@ -193,12 +307,10 @@ __global__ void __launch_bounds__(kBulkNT, 2) ds_label_bulk_kernel(const TKV* __
                 }
             }
         }
-        __syncthreads();  // every thread is done with the slot
-        if (!__syncthreads_and(ok)) break;  // a copy never arrived: leave (recorded in *err)
-        if (tid == 0) {
-            const long long nx = it + (long long)kBulkStages * gridDim.x;
-            if (nx < items) issue(nx, slot);
-        }
+        // every thread is done with the slot; a copy that never arrived
+        // (recorded in *err) ends the CTA
+        if (!__syncthreads_and(ok)) break;
+        if (tid == 0 && pit < items) issue(slot);
     }
 }
 
@@ -213,7 +325,7 @@ static cudaError_t launch_label_bulk(const LabelArgs& a, long long items, cudaSt
     }
     const long long grid = items < 2LL * a.sms ? items : 2LL * a.sms;
     ds_label_bulk_kernel<TKV, LK, D, CI><<<(unsigned)grid, kBulkNT, bulk_smem_bytes(), st>>>(
-        reinterpret_cast<const TKV*>(a.k), a.idx, a.hkv, a.t_begin, a.t_end, a.s_cap, a.c, a.b * a.hkv,
+        reinterpret_cast<const TKV*>(a.k), a.idx, a.hkv, a.t_begin, a.t_end, a.s_cap, a.b * a.hkv,
         reinterpret_cast<uint8_t*>(a.label), a.lscale, a.lzero, a.err);
     return cudaGetLastError();
 }
@@ -223,8 +335,8 @@ static cudaError_t launch_label_t(const LabelArgs& a, cudaStream_t st) {
     const int n = a.t_end - a.t_begin;
     constexpr int kTok = kBulkStage / (D * Elem<TKV>::kBytes);
     const long long items = (long long)a.b * a.hkv * ((n + kTok - 1) / kTok);
-    if (!a.block_table && a.err && items >= 2 * (long long)a.sms && (LK == 0 || a.c >= 2 * kPackLanes)) {
-        if constexpr (LK == 0) return launch_label_bulk<TKV, 0, D, 0>(a, items, st);
+    if (!a.block_table && a.err && items >= 2 * (long long)a.sms && items < (1LL << 30) &&
+        (LK == 0 || a.c >= 2 * kPackLanes)) {
         switch (a.c) {
         case 8: return launch_label_bulk<TKV, LK, D, 8>(a, items, st);
         case 16: return launch_label_bulk<TKV, LK, D, 16>(a, items, st);

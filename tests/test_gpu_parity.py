@@ -157,6 +157,35 @@ def test_pipelined_label_build_bit_exact(kv, label, d, c):
         assert torch.all(lab[:, :, wl.s:] == 3)
 
 
+@pytest.mark.parametrize("kv,c", [("bf16", 32), ("f32", 16), ("bf16", 64)])
+def test_pipelined_int4_half_way_codes(kv, c):
+    """4-bit prefill build where many quotients (x - zero) / scale are exact
+    half-integers: each heavy row spans [0, 15 h] with h a power of two, so
+    scale = h exactly and odd multiples of h / 2 sit half-way between two
+    codes. Rounding must be half to even, as the IEEE quotient gives; the
+    kernel's reciprocal shortcut has to fall back to the division there."""
+    wl = synth.custom(b=4, hq=8, hkv=8, d=128, s=1000, c=c, kv_dtype=kv, label_dtype="int4",
+                      n_outlier=min(8, c), index=67)
+    di = synth.decode_inputs(wl, s_cap=1000)
+    idx = _idx_random(wl, 11)
+    r = np.random.default_rng(5)
+    k = synth.storage_to_f32(di.k, kv).copy()
+    for g in range(wl.hkv):
+        h = 2.0 ** r.integers(-4, 3, size=(wl.b, wl.s))
+        m = r.integers(0, 31, size=(wl.b, wl.s, c)).astype(np.float64)  # multiples of h / 2 in [0, 15 h]
+        m[:, :, 0], m[:, :, 1] = 0, 30
+        k[:, g, :, idx[g]] = np.moveaxis(m * h[:, :, None] / 2, 2, 0)
+    kst = synth.to_storage(k.astype(np.float32), kv)
+    assert np.array_equal(synth.storage_to_f32(kst, kv), k.astype(np.float32))  # exact in the key dtype
+    kd, idxd = to_dev(kst, kv), torch.from_numpy(idx).cuda()
+    lab, sc, ze = _gpu_label(kd, idxd, wl.s, wl)
+    ds.check_device()
+    got = _host_label(lab, sc, ze, wl)
+    ref = oracle.build_label(kst, kv, "int4", idx, wl.s)
+    for a, b_ in zip(got, ref):
+        assert np.array_equal(a, b_)
+
+
 def test_bounded_wait_self_test_reports_timeout():
     """A kernel wait that runs out is recorded and reported, and the context
     stays usable: a transaction barrier nothing completes, waited on for about
