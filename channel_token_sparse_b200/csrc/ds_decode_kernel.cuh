@@ -280,7 +280,16 @@ __device__ __forceinline__ void cluster_select_bin(cg::cluster_group& cluster, u
     const int tid = threadIdx.x;
     const int bin = 255 - tid;  // thread 0 holds the largest bin
     uint32_t cnt = 0;
-    for (int r = 0; r < nblocks; ++r) cnt += row_smem(cluster, nblocks, hist, r)[bin];
+    if (nblocks == 1) {
+        cnt = hist[bin];
+    } else {
+        // all remote loads in flight together, then the sum
+        uint32_t v[kMaxCluster];
+#pragma unroll
+        for (int r = 0; r < kMaxCluster; ++r) v[r] = r < nblocks ? cluster.map_shared_rank(hist, r)[bin] : 0u;
+#pragma unroll
+        for (int r = 0; r < kMaxCluster; ++r) cnt += v[r];
+    }
     if (zero_next) zero_next[tid] = 0u;
     // prefix over bins (largest first): warp scans, then every warp adds the
     // totals of the warps before it (one barrier, no second scan)
