@@ -77,7 +77,8 @@ __global__ void __launch_bounds__(kLabNT) ds_label_kernel(const TKV* __restrict_
 // in), so the next blocks' reads are in flight while the current one is
 // gathered or packed. Same results as ds_label_kernel.
 constexpr int kBulkStage = 16384;  // bytes of key rows per stage
-constexpr int kBulkStages = 6;
+constexpr int kBulkStages = 4;
+constexpr int kBulkCtasPerSm = 3;  // 3 x (4 x 16 KiB) of ring per SM; <= 85 registers
 constexpr int kBulkNT = 256;
 // packing threads per token (4-bit): each takes c / kPackLanes channels
 constexpr int kPackLanes = 4;
@@ -115,27 +116,29 @@ struct ItemCursor {
 };
 
 // 4-bit codes of n values a_e = x_e - zero: the quotient a_e / scale is
-// formed with the rounded reciprocal, and only where it lies within 1e-5 of a
-// half-integer (where the two could round differently) is it recomputed with
-// the IEEE division; rint (half to even) then clamp to [0, 15], which
-// __float2int_rn followed by an integer clamp gives for every input (NaN
-// converts to 0). The codes equal those of int4_code.
+// formed with the rounded reciprocal and rounded to an integer r (half to
+// even); only where it lies within about 1e-5 of a half-integer (|q - r| near
+// 0.5, where the product and the IEEE quotient could round differently) is it
+// recomputed with the IEEE division. The code is r clamped to [0, 15] (NaN
+// gives 0); the codes equal those of int4_code.
 template <int N>
 __device__ __forceinline__ void int4_codes(const float (&a)[N], float sc, float rcp_sc, uint32_t (&code)[N]) {
-    float q[N];
+    float r[N];
     uint32_t near = 0u;
 #pragma unroll
     for (int e = 0; e < N; ++e) {
-        q[e] = __fmul_rn(a[e], rcp_sc);
-        if (fabsf(q[e] - floorf(q[e]) - 0.5f) <= 1e-5f) near |= 1u << e;
+        const float q = __fmul_rn(a[e], rcp_sc);
+        r[e] = rintf(q);
+        if (fabsf(q - r[e]) >= 0.5f - 1e-5f) near |= 1u << e;
     }
     if (near) {
 #pragma unroll
         for (int e = 0; e < N; ++e)
-            if ((near >> e) & 1u) q[e] = __fdiv_rn(a[e], sc);
+            if ((near >> e) & 1u) r[e] = rintf(__fdiv_rn(a[e], sc));
     }
 #pragma unroll
-    for (int e = 0; e < N; ++e) code[e] = sc > 0.f ? (uint32_t)min(max(__float2int_rn(q[e]), 0), 15) : 0u;
+    for (int e = 0; e < N; ++e)
+        code[e] = sc > 0.f ? (uint32_t)fminf(fmaxf(r[e], 0.f), 15.f) : 0u;
 }
 
 // Pick element (p - r) & 3 of a: the value a rotated thread read for output
@@ -159,7 +162,7 @@ __device__ __forceinline__ uint32_t pick_rot(const uint32_t (&a)[4], int p, int 
 // is that of pack_int4_row, with mn / mx combined over the lanes (fminf /
 // fmaxf do not depend on the order).
 template <typename TKV, int LK, int D, int CI>
-__global__ void __launch_bounds__(kBulkNT, 2) ds_label_bulk_kernel(const TKV* __restrict__ k,
+__global__ void __launch_bounds__(kBulkNT, kBulkCtasPerSm) ds_label_bulk_kernel(const TKV* __restrict__ k,
                                                                   const int32_t* __restrict__ idx, int hkv,
                                                                   int t_begin, int t_end, int s_cap, int rows,
                                                                   uint8_t* __restrict__ label,
@@ -323,7 +326,8 @@ static cudaError_t launch_label_bulk(const LabelArgs& a, long long items, cudaSt
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    const long long grid = items < 2LL * a.sms ? items : 2LL * a.sms;
+    const long long slots = (long long)kBulkCtasPerSm * a.sms;
+    const long long grid = items < slots ? items : slots;
     ds_label_bulk_kernel<TKV, LK, D, CI><<<(unsigned)grid, kBulkNT, bulk_smem_bytes(), st>>>(
         reinterpret_cast<const TKV*>(a.k), a.idx, a.hkv, a.t_begin, a.t_end, a.s_cap, a.b * a.hkv,
         reinterpret_cast<uint8_t*>(a.label), a.lscale, a.lzero, a.err);
@@ -335,7 +339,7 @@ static cudaError_t launch_label_t(const LabelArgs& a, cudaStream_t st) {
     const int n = a.t_end - a.t_begin;
     constexpr int kTok = kBulkStage / (D * Elem<TKV>::kBytes);
     const long long items = (long long)a.b * a.hkv * ((n + kTok - 1) / kTok);
-    if (!a.block_table && a.err && items >= 2 * (long long)a.sms && items < (1LL << 30) &&
+    if (!a.block_table && a.err && items >= (long long)kBulkCtasPerSm * a.sms && items < (1LL << 30) &&
         (LK == 0 || a.c >= 2 * kPackLanes)) {
         switch (a.c) {
         case 8: return launch_label_bulk<TKV, LK, D, 8>(a, items, st);
