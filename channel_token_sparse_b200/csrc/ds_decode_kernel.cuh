@@ -1097,18 +1097,25 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
             const int stages = p.att_stages;
             uint8_t* ring = smem + L.region + wid * att_ring_bytes(RB, 2, stages);
             const int nb = n_att > wid * TB8 ? (n_att - wid * TB8 + kNW * TB8 - 1) / (kNW * TB8) : 0;
+            // lane l copies 16-byte chunk l % kChunks of token rows l / kChunks,
+            // l / kChunks + 32 / kChunks, ... of the tile, the K and the V row of
+            // each token together (one row lookup per token)
+            static_assert(32 % kChunks == 0 && TB8 % (32 / kChunks) == 0, "chunk layout");
+            constexpr int kRowsPerPass = 32 / kChunks;
+            const int cl = lane % kChunks, ul = lane / kChunks;
             auto issue_stage = [&](int bi) {
                 const int bt0 = (wid + bi * kNW) * TB8;
                 uint8_t* st = ring + (bi % stages) * kStageBytes;
     #pragma unroll
-                for (int pc = lane; pc < 2 * TB8 * kChunks; pc += 32) {
-                    const int r = pc / kChunks, c = pc - r * kChunks;
-                    const int u = r & (TB8 - 1);
+                for (int u0 = 0; u0 < TB8; u0 += kRowsPerPass) {
+                    const int u = u0 + ul;
                     const bool ok = bt0 + u < n_att;
-                    const TKV* base = r < TB8 ? kb : vb;
-                    const TKV* src = ok ? base + att_row(bt0 + u) * D : base;
+                    const size_t off = ok ? att_row(bt0 + u) * D : 0;
+                    const uint8_t* ks = reinterpret_cast<const uint8_t*>(kb + off) + (cl << 4);
+                    const uint8_t* vs = reinterpret_cast<const uint8_t*>(vb + off) + (cl << 4);
                     // rows of tokens past the end are zero-filled (their p is 0, and 0 * garbage could be NaN)
-                    cp_async16_zfill(st + r * RB + ((c ^ u) << 4), reinterpret_cast<const uint8_t*>(src) + (c << 4), ok);
+                    cp_async16_zfill(st + u * RB + ((cl ^ u) << 4), ks, ok);
+                    cp_async16_zfill(st + (TB8 + u) * RB + ((cl ^ u) << 4), vs, ok);
                 }
             };
             for (int bi = 0; bi < stages - 1; ++bi) {
@@ -1151,19 +1158,27 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
                 float mx = fmaxf(z0, z1);
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                const float m_new = fmaxf(m_run, mx);
-                const float corr = exp2f(m_run - m_new);
+                // The running max moves only when the tile's max exceeds it by
+                // more than 2^kSlack (probabilities then stay below 2^kSlack): most
+                // tiles leave it, and the rescale of O, alone. O and l share the
+                // same max, so O / l is unchanged.
+                constexpr float kSlack = 8.f;
+                const bool move = mx > m_run + kSlack;
+                const float m_new = move ? mx : m_run;
+                const float corr = move ? exp2f(m_run - m_new) : 1.f;
                 const float p0 = exp2f(z0 - m_new), p1 = exp2f(z1 - m_new);
                 float rs = p0 + p1;
                 rs += __shfl_xor_sync(0xffffffffu, rs, 1);
                 rs += __shfl_xor_sync(0xffffffffu, rs, 2);
                 l_run = l_run * corr + rs;
                 m_run = m_new;
-                // O^T columns are heads kc, kc + 1: fetch their corrections
-                const float ca = __shfl_sync(0xffffffffu, corr, 4 * kc);
-                const float cb = __shfl_sync(0xffffffffu, corr, 4 * kc + 4);
+                if (__any_sync(0xffffffffu, move)) {
+                    // O^T columns are heads kc, kc + 1: fetch their corrections
+                    const float ca = __shfl_sync(0xffffffffu, corr, 4 * kc);
+                    const float cb = __shfl_sync(0xffffffffu, corr, 4 * kc + 4);
     #pragma unroll
-                for (int i = 0; i < D / 16; ++i) { o[i][0] *= ca; o[i][1] *= cb; o[i][2] *= ca; o[i][3] *= cb; }
+                    for (int i = 0; i < D / 16; ++i) { o[i][0] *= ca; o[i][1] *= cb; o[i][2] *= ca; o[i][3] *= cb; }
+                }
                 const uint32_t ph = pack_bf16x2(p0, p1);
                 const uint32_t pl = pack_bf16x2(p0 - bf16lo(ph), p1 - bf16hi(ph));
                 // O^T += V^T P^T; one ldmatrix.x4.trans covers two 16-dim row tiles

@@ -123,22 +123,24 @@ struct ItemCursor {
 // gives 0); the codes equal those of int4_code.
 template <int N>
 __device__ __forceinline__ void int4_codes(const float (&a)[N], float sc, float rcp_sc, uint32_t (&code)[N]) {
+    constexpr float kNear = 0.5f - 1e-5f;
     float r[N];
-    uint32_t near = 0u;
+    bool near = false;
 #pragma unroll
     for (int e = 0; e < N; ++e) {
         const float q = __fmul_rn(a[e], rcp_sc);
         r[e] = rintf(q);
-        if (fabsf(q - r[e]) >= 0.5f - 1e-5f) near |= 1u << e;
+        near |= fabsf(q - r[e]) >= kNear;
     }
     if (near) {
 #pragma unroll
-        for (int e = 0; e < N; ++e)
-            if ((near >> e) & 1u) r[e] = rintf(__fdiv_rn(a[e], sc));
+        for (int e = 0; e < N; ++e) {
+            const float q = __fmul_rn(a[e], rcp_sc);
+            if (fabsf(q - rintf(q)) >= kNear) r[e] = rintf(__fdiv_rn(a[e], sc));
+        }
     }
 #pragma unroll
-    for (int e = 0; e < N; ++e)
-        code[e] = sc > 0.f ? (uint32_t)fminf(fmaxf(r[e], 0.f), 15.f) : 0u;
+    for (int e = 0; e < N; ++e) code[e] = (uint32_t)fminf(fmaxf(r[e], 0.f), 15.f);
 }
 
 // Pick element (p - r) & 3 of a: the value a rotated thread read for output
@@ -285,19 +287,38 @@ __global__ void __launch_bounds__(kBulkNT, kBulkCtasPerSm) ds_label_bulk_kernel(
                         for (int e = 0; e < kPer; ++e) a[e] = __fsub_rn(v[e], z);
                         uint32_t code[kPer];
                         int4_codes<kPer>(a, sc, rsc, code);
+                        if (!(sc > 0.f)) {
+#pragma unroll
+                            for (int e = 0; e < kPer; ++e) code[e] = 0u;
+                        }
                         // channel q4 * kPer + e of the row is nibble e of this
                         // lane's kPer / 2 bytes (low nibble first)
                         uint8_t* dst = label + (tok0 + t) * (size_t)(CI / 2) + q4 * kPer / 2;
                         if constexpr (kRot) {
+                            // the codes in the rotated order, packed, then the
+                            // word rotated left by 4 * rot bits (nibble e to
+                            // nibble (e + rot) % kPer)
                             uint64_t w = 0;
 #pragma unroll
-                            for (int e = 0; e < kPer; ++e) w |= (uint64_t)code[e] << (4 * ((e + rot) % kPer));
+                            for (int e = 0; e < kPer; ++e) w |= (uint64_t)code[e] << (4 * e);
+                            const uint32_t sh = 4u * (uint32_t)rot;
                             // dst is kPer / 2-byte aligned: label is 16-byte
                             // aligned and rows are 2 * kPer bytes long
-                            if constexpr (kPer == 2) *dst = (uint8_t)w;
-                            else if constexpr (kPer == 4) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)w;
-                            else if constexpr (kPer == 8) *reinterpret_cast<uint32_t*>(dst) = (uint32_t)w;
-                            else *reinterpret_cast<uint64_t*>(dst) = w;
+                            if constexpr (kPer == 2) {
+                                const uint32_t x = (uint32_t)w * 0x101u;  // the byte twice
+                                *dst = (uint8_t)(x >> (8u - sh));
+                            } else if constexpr (kPer == 4) {
+                                const uint32_t x = (uint32_t)w * 0x10001u;
+                                *reinterpret_cast<uint16_t*>(dst) = (uint16_t)(x >> (16u - sh));
+                            } else if constexpr (kPer == 8) {
+                                *reinterpret_cast<uint32_t*>(dst) = __funnelshift_l((uint32_t)w, (uint32_t)w, sh);
+                            } else {
+                                const uint32_t lo = (uint32_t)w, hi = (uint32_t)(w >> 32);
+                                const uint32_t l2 = sh >= 32u ? hi : lo, h2 = sh >= 32u ? lo : hi;
+                                const uint32_t s2 = sh & 31u;
+                                *reinterpret_cast<uint2*>(dst) =
+                                    make_uint2(__funnelshift_l(h2, l2, s2), __funnelshift_l(l2, h2, s2));
+                            }
                         } else {
 #pragma unroll
                             for (int e = 0; e < kPer; e += 2) dst[e / 2] = (uint8_t)(code[e] | (code[e + 1] << 4));
