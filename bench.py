@@ -48,6 +48,7 @@ CHAIN_STEPS = 8  # at least this many consecutive steps per captured graph
 KERNEL_SOURCES = ["channel_token_sparse_b200/csrc/ds_decode_kernel.cuh",
                   "channel_token_sparse_b200/csrc/ds_common.cuh",
                   "channel_token_sparse_b200/csrc/ds_decode_bf16_fp.cu",
+                  "channel_token_sparse_b200/csrc/ds_decode_bf16_i4.cu",
                   "channel_token_sparse_b200/csrc/ds_api.cu"]
 
 

@@ -514,8 +514,9 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     }
     // decode step: the CTA holding token s-1 builds its label row (the same
     // copy / 4-bit pack as ds_append_label), keeps it in shared memory and
-    // stores it to the label cache
-    if (app_i >= 0 && wid == 0) {
+    // stores it to the label cache; 4-bit rows use warp 1, so the pack runs
+    // beside warp 0's fixed-point limbs
+    if (app_i >= 0 && wid == (LK == kLabelInt4 ? 1 : 0)) {
         const TKV* krow = reinterpret_cast<const TKV*>(krow_s);
         uint8_t* grow = const_cast<uint8_t*>(lab) + (size_t)(s - 1) * LG::kBytes;
         if constexpr (LK == kLabelFp) {
@@ -526,15 +527,21 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
                 reinterpret_cast<TKV*>(grow)[j] = x;
             }
         } else {
-            // pack_int4_row's arithmetic with a lane per channel: every lane
-            // forms mn / mx in channel order (as the serial form does), then
-            // lane j divides for channel j and the even lanes pack pairs
+            // pack_int4_row's arithmetic with a lane per channel: mn / mx by a
+            // butterfly over the lanes (fminf / fmaxf do not depend on the
+            // order), then lane j divides for channel j and the even lanes
+            // pack pairs
             uint16_t* ssz = reinterpret_cast<uint16_t*>(smem + L.app + align16(C * 4));
-            float mn = Elem<TKV>::to_f32(krow[idx_s[0]]), mx = mn;
-            for (int j = 1; j < C; ++j) {
+            float mn = Elem<TKV>::to_f32(krow[idx_s[lane % C]]), mx = mn;
+            for (int j = lane + 32; j < C; j += 32) {
                 const float v = Elem<TKV>::to_f32(krow[idx_s[j]]);
                 mn = fminf(mn, v);
                 mx = fmaxf(mx, v);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
             }
             const float step = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
             const uint16_t sh = __half_as_ushort(__float2half_rn(step));
