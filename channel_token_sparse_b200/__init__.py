@@ -184,7 +184,7 @@ def check_device(stream=None) -> None:
 
 
 def tune(name: str, value: int) -> None:
-    """Set a decode tuning knob ("stagger", "att_prefetch", "scan_prefetch");
+    """Set a decode tuning knob ("scan_prefetch", "i4_ring", "list_path");
     a negative value restores its default."""
     _check(lib().ds_sparse_decode_tune(name.encode(), int(value)))
 
