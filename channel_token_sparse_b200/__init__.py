@@ -184,7 +184,7 @@ def check_device(stream=None) -> None:
 
 
 def tune(name: str, value: int) -> None:
-    """Set a decode tuning knob ("scan_prefetch", "i4_ring", "list_path");
+    """Set a decode tuning knob ("scan_prefetch", "i4_ring");
     a negative value restores its default."""
     _check(lib().ds_sparse_decode_tune(name.encode(), int(value)))
 
