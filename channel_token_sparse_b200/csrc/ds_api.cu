@@ -565,7 +565,7 @@ ds_status ds_sparse_decode_plan(int b, int hq, int hkv, int s, int d, int c, int
     Plan pl;
     if (!make_plan(b * hkv, hq / hkv, s, d, c, topk, false, label_dt == DS_INT4, kvdt == DS_F32 ? 4 : 2,
                    kCtasPerSm * 148,
-                   g_cluster_override.load(), &pl))
+                   g_cluster_override.load(), &pl, s))
         return fail(DS_ERR_UNSUPPORTED, "no feasible launch plan (s too long for 16 CTAs per row)");
     if (cluster_out) *cluster_out = pl.N;
     if (chunk_out) *chunk_out = pl.chunk;

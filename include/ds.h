@@ -308,9 +308,10 @@ DS_API ds_status ds_decode_step_paged(const void* q, const void* k_pool, const v
                                       int topk, float sm_scale, void* out, ds_dtype out_dt,
                                       int32_t* sel_out, float* score_out, cudaStream_t stream);
 
-/* Launch plan of ds_sparse_decode for a shape (host only, launches nothing):
- * CTAs per thread-block cluster (one cluster per (b, kv head)), tokens per
- * CTA and dynamic shared memory per CTA in bytes. Any output may be NULL. */
+/* Launch plan of ds_sparse_decode for a shape (host only, launches nothing),
+ * for caches of capacity s on a 148-SM B200: CTAs per thread-block cluster
+ * (one cluster per (b, kv head)), tokens per CTA and dynamic shared memory
+ * per CTA in bytes. Any output may be NULL. */
 DS_API ds_status ds_sparse_decode_plan(int b, int hq, int hkv, int s, int d, int c, int topk,
                                 ds_dtype kvdt, ds_dtype label_dt,
                                 int* cluster_out, int* chunk_out, int* smem_out);
