@@ -113,9 +113,10 @@ __host__ __device__ inline int sel_scratch_bytes(int chunk);
 // (at most 8 * (128 + 2) floats) is later written into its own ring.
 constexpr int kAttStagesF32 = 4;
 // Label-streaming ring (fp labels): stages of one row per thread.
-// Stages of the label ring (8 for both kinds: a 12-stage ring for the short
-// 4-bit rows was measured no faster).
-__host__ __device__ constexpr int lab_stages(bool) { return 8; }
+// Stages of the label ring: 8 for fp rows; 6 for 4-bit rows, whose ring
+// then fits beside the kept low key bits on the 32-channel layer (12 stages
+// were measured no faster than 8, 6 slightly faster).
+__host__ __device__ constexpr int lab_stages(bool int4) { return int4 ? 6 : 8; }
 // ring bytes for label rows of `label_row_bytes` (a 4-bit row adds its fp16
 // scale and zero, 4 bytes, kept in two arrays of the stage)
 __host__ __device__ constexpr int lab_ring_bytes(int label_row_bytes, bool int4) {
@@ -412,6 +413,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     // 0..7 of that warp (so a __syncwarp makes them visible to its lanes).
     constexpr bool kI4 = LK == kLabelInt4;
     constexpr int kLabStages = lab_stages(kI4);
+    static_assert(kLabStages % 2 == 0 && kLabStages >= 4, "the scan takes two stages per iteration");
     constexpr bool kRingable = kI4 ? (LG::kBytes == 4 || LG::kBytes == 8 || LG::kBytes % 16 == 0)
                                    : LG::kBytes % 16 == 0;
     const bool use_ring = kRingable && need_scores && p.lab_ring;
@@ -420,10 +422,13 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     constexpr int kSlot = LG::kBytes;               // payload bytes per token
     constexpr int kStage = kNT * (kSlot + (kI4 ? 4 : 0));
     const int nst = (n_loc + kNT - 1) / kNT;
-    auto issue = [&](int j) {
+    // stage j goes to ring slot `slot` (= j mod kLabStages, kept by the
+    // caller); i < n_loc implies j < nst. The appended token's row is copied
+    // too (stale, never read: stage_row takes it from shared memory).
+    auto issue = [&](int j, int slot) {
         const int i = j * kNT + tid;
-        uint8_t* stg = lring + (j % kLabStages) * kStage;
-        if (j < nst && i < n_loc && i != app_i) {
+        uint8_t* stg = lring + slot * kStage;
+        if (i < n_loc) {
             uint8_t* dst = stg + tid * kSlot;
             const uint8_t* src = lab + (size_t)(t0 + i) * kSlot;
             if constexpr (kSlot % 16 == 0) {
@@ -437,7 +442,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
         }
         if constexpr (kI4) {
             const int c8 = (wid * 32 + (lane & 3) * 8);   // first token of this lane's chunk
-            if (j < nst && lane < 8 && j * kNT + c8 < n_loc) {
+            if (lane < 8 && j * kNT + c8 < n_loc) {
                 const uint16_t* src = (lane < 4 ? lsc : lze) + t0 + j * kNT + c8;
                 uint8_t* dst = stg + kNT * kSlot + (lane < 4 ? 0 : kNT * 2) + c8 * 2;
                 cp_async16(dst, src);
@@ -446,7 +451,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     };
     if (use_ring) {
 #pragma unroll 1
-        for (int j = 0; j < kLabStages - 2; ++j) { issue(j); cp_async_commit(); }
+        for (int j = 0; j < kLabStages - 2; ++j) { issue(j, j); cp_async_commit(); }
     }
 
 #pragma unroll
@@ -649,33 +654,35 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     if (use_ring) {
         // two stages per iteration: each thread scores two tokens (j and
         // j + 1 stages apart) whose arithmetic chains are independent
-        auto stage_row = [&](int j, int i, uint32_t (&w)[LG::kWords], float& ss, float& zz) {
-            const uint8_t* stg = lring + (j % kLabStages) * kStage;
-            if (i == app_i) {
-                lds_row<LG::kBytes>(w, app_row);
-                if constexpr (kI4) { ss = fp16_bits_to_f32(app_sz[0]); zz = fp16_bits_to_f32(app_sz[1]); }
-            } else {
-                lds_row<LG::kBytes>(w, stg + tid * kSlot);
-                if constexpr (kI4) {
-                    ss = fp16_bits_to_f32(reinterpret_cast<const uint16_t*>(stg + kNT * kSlot)[tid]);
-                    zz = fp16_bits_to_f32(reinterpret_cast<const uint16_t*>(stg + kNT * kSlot + kNT * 2)[tid]);
-                }
+        // the row of local token i from ring slot `slot` (the appended token's
+        // from shared memory): pointers picked, no branch
+        auto stage_row = [&](int slot, int i, uint32_t (&w)[LG::kWords], float& ss, float& zz) {
+            const uint8_t* stg = lring + slot * kStage;
+            const bool app = i == app_i;
+            lds_row<LG::kBytes>(w, app ? app_row : stg + tid * kSlot);
+            if constexpr (kI4) {
+                const uint16_t* sp = app ? app_sz : reinterpret_cast<const uint16_t*>(stg + kNT * kSlot) + tid;
+                ss = fp16_bits_to_f32(sp[0]);
+                zz = fp16_bits_to_f32(sp[app ? 1 : kNT]);
             }
         };
+        int sj = 0;  // ring slot of stage j (j even; kLabStages is even)
 #pragma unroll 1
         for (int j = 0; j < nst; j += 2) {
             if constexpr (kI4) __syncwarp();   // every lane is done with the slots refilled next
-            issue(j + kLabStages - 2);
+            const int sr = sj == 0 ? kLabStages - 2 : sj - 2;   // slot of stage j + kLabStages - 2
+            issue(j + kLabStages - 2, sr);
             cp_async_commit();
-            issue(j + kLabStages - 1);
+            issue(j + kLabStages - 1, sr + 1);
             cp_async_commit();
             cp_async_wait<kLabStages - 2>();   // stages j and j + 1 have landed
             if constexpr (kI4) __syncwarp();   // the warp's scale / zero chunks
             const int i0 = j * kNT + tid, i1 = i0 + kNT;
             uint32_t w0[LG::kWords], w1[LG::kWords];
             float ss0 = 0.f, zz0 = 0.f, ss1 = 0.f, zz1 = 0.f;
-            stage_row(j, i0, w0, ss0, zz0);
-            stage_row(j + 1, i1, w1, ss1, zz1);
+            stage_row(sj, i0, w0, ss0, zz0);
+            stage_row(sj + 1, i1, w1, ss1, zz1);
+            sj = sj + 2 == kLabStages ? 0 : sj + 2;
             // rows past the chunk hold stale ring bytes: scored, not recorded
             const float sv0 = label_score<TKV, LK, C>(w0, qreg, qLs, ss0, zz0, qsum, lim, s_e);
             const float sv1 = label_score<TKV, LK, C>(w1, qreg, qLs, ss1, zz1, qsum, lim, s_e);
