@@ -1117,9 +1117,11 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
             static_assert(32 % kChunks == 0 && TB8 % (32 / kChunks) == 0, "chunk layout");
             constexpr int kRowsPerPass = 32 / kChunks;
             const int cl = lane % kChunks, ul = lane / kChunks;
-            auto issue_stage = [&](int bi) {
+            // tile bi of this warp goes to ring slot `slot` (= bi mod stages,
+            // kept by the caller: stages is a launch parameter)
+            auto issue_stage = [&](int bi, int slot) {
                 const int bt0 = (wid + bi * kNW) * TB8;
-                uint8_t* st = ring + (bi % stages) * kStageBytes;
+                uint8_t* st = ring + slot * kStageBytes;
     #pragma unroll
                 for (int u0 = 0; u0 < TB8; u0 += kRowsPerPass) {
                     const int u = u0 + ul;
@@ -1133,7 +1135,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
                 }
             };
             for (int bi = 0; bi < stages - 1; ++bi) {
-                if (bi < nb) issue_stage(bi);
+                if (bi < nb) issue_stage(bi, bi);
                 cp_async_commit();
             }
             // Q fragments (A operand, rows = heads): bf16 pairs, exact (q is bf16),
@@ -1145,14 +1147,16 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
             for (int i = 0; i < D / 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
             float m_run = -INFINITY, l_run = 0.f;  // for head hr (row of Z)
             // [phase] 21
+            int cs = 0;  // ring slot of tile bi
     #pragma unroll 1
             for (int bi = 0; bi < nb; ++bi) {
-                if (bi + stages - 1 < nb) issue_stage(bi + stages - 1);
+                if (bi + stages - 1 < nb) issue_stage(bi + stages - 1, cs == 0 ? stages - 1 : cs - 1);
                 cp_async_commit();
                 if (stages == 3) cp_async_wait<2>();
                 else cp_async_wait<1>();
                 __syncwarp();
-                const uint8_t* st = ring + (bi % stages) * kStageBytes;
+                const uint8_t* st = ring + cs * kStageBytes;
+                cs = cs + 1 == stages ? 0 : cs + 1;
                 const int bt0 = (wid + bi * kNW) * TB8;
                 // Z = Q K^T over D in 16-dim steps; one ldmatrix.x4 covers 32 dims
                 float z[4] = {0.f, 0.f, 0.f, 0.f};
