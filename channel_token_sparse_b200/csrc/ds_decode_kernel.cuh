@@ -425,12 +425,17 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
     // stage j goes to ring slot `slot` (= j mod kLabStages, kept by the
     // caller); i < n_loc implies j < nst. The appended token's row is copied
     // too (stale, never read: stage_row takes it from shared memory).
+    // per-thread bases of the copies; stage j adds j * kNT tokens
+    const uint8_t* lab_t = lab + (size_t)(t0 + tid) * kSlot;
+    uint8_t* ring_t = lring + tid * kSlot;
+    const int c8 = wid * 32 + (lane & 3) * 8;   // 4-bit: first token of this lane's scale / zero chunk
+    const uint16_t* sz_t = kI4 ? (lane < 4 ? lsc : lze) + t0 + c8 : nullptr;
+    const int sz_off = kNT * kSlot + (lane < 4 ? 0 : kNT * 2) + c8 * 2;
     auto issue = [&](int j, int slot) {
-        const int i = j * kNT + tid;
-        uint8_t* stg = lring + slot * kStage;
-        if (i < n_loc) {
-            uint8_t* dst = stg + tid * kSlot;
-            const uint8_t* src = lab + (size_t)(t0 + i) * kSlot;
+        const int jr = j * kNT;
+        if (jr + tid < n_loc) {
+            uint8_t* dst = ring_t + slot * kStage;
+            const uint8_t* src = lab_t + (size_t)jr * kSlot;
             if constexpr (kSlot % 16 == 0) {
 #pragma unroll
                 for (int o = 0; o < kSlot; o += 16) cp_async16(dst + o, src + o);
@@ -441,12 +446,7 @@ __global__ void __launch_bounds__(kNT, 2) ds_decode_kernel(const DecodeParams p)
             }
         }
         if constexpr (kI4) {
-            const int c8 = (wid * 32 + (lane & 3) * 8);   // first token of this lane's chunk
-            if (lane < 8 && j * kNT + c8 < n_loc) {
-                const uint16_t* src = (lane < 4 ? lsc : lze) + t0 + j * kNT + c8;
-                uint8_t* dst = stg + kNT * kSlot + (lane < 4 ? 0 : kNT * 2) + c8 * 2;
-                cp_async16(dst, src);
-            }
+            if (lane < 8 && jr + c8 < n_loc) cp_async16(lring + slot * kStage + sz_off, sz_t + jr);
         }
     };
     if (use_ring) {
