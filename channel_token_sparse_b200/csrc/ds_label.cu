@@ -5,9 +5,13 @@
 // contiguous label cache; at each decode step only the new token's channels
 // are added. The cache may be kept in 4 bits.
 //
-// One CTA handles kTokens consecutive tokens of one (b, kv head) row: the key
-// rows are staged in shared memory with coalesced 16-byte loads, then each
-// label element (fp) or each token (4-bit) is produced from shared memory.
+// Two kernels. Prefill builds over a dense key cache with enough work for
+// every resident CTA run ds_label_bulk_kernel: persistent CTAs stream 16 KiB
+// blocks of key rows through a shared-memory ring filled by 1-D bulk copies.
+// Appends, paged caches and small builds run ds_label_kernel: one CTA
+// handles kTokens consecutive tokens of one (b, kv head) row, staging the key
+// rows in shared memory with coalesced 16-byte loads. Both then produce each
+// label element (fp) or each token's 4-bit codes from shared memory.
 // The key cache is dense [b, hkv, s_cap, d] or paged (a block table maps
 // token t of entry b to a row of a [num_blocks, hkv, page, d] pool); the
 // label cache is always dense [b, hkv, s_cap, c].
