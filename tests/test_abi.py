@@ -108,6 +108,13 @@ def test_plan_choices(lib):
     assert (n, chunk) == (8, 32768) and smem <= 227 * 1024
     n, chunk, _ = ds.plan(1, 2, 2, 512, 64, 8, 32, ds.DS_F32, ds.DS_F32)
     assert n * chunk >= 512 and chunk >= 256
+    # the four benchmark layers keep two CTAs per SM: (228 KiB - 2 KiB) / 2 of
+    # shared memory each at most
+    for shape in ((8, 32, 32, 4096, 128, 16, 256, ds.DS_BF16, ds.DS_BF16),
+                  (32, 32, 32, 16384, 128, 32, 1024, ds.DS_BF16, ds.DS_INT4),
+                  (4, 32, 8, 32768, 128, 16, 2048, ds.DS_BF16, ds.DS_BF16),
+                  (1, 32, 32, 262144, 128, 16, 16384, ds.DS_BF16, ds.DS_BF16)):
+        assert ds.plan(*shape)[2] <= (228 - 2) * 1024 // 2, shape
     ds.set_cluster(16)
     try:
         assert ds.plan(8, 32, 32, 4096, 128, 16, 256)[:2] == (16, 256)
